@@ -1,0 +1,392 @@
+#!/usr/bin/env python3
+"""Benchmark: the loss-scaled FP32-master optimizer step (libmpt) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl mpt|reference]
+                    [--workload gpt2_medium]
+
+One step = one mpt_step call over the whole parameter list: the check kernel
+(overflow flag, range counts, global sum of squares) and the fused update
+kernel (unscale, global-L2 clip, weight decay, momentum, FP32 master, FP16
+copy), plus the 80-byte result read-back the call makes.  The workload is the
+GPT-2-medium-shaped list (292 tensors, 354 823 168 parameters, clip 1.0): the
+first of the workloads at >= 100M parameters, the size the 80%-of-HBM target
+is set at.  Inputs are seeded synthetic FP16 gradients (two sets, alternated)
+and random-initialised FP32 masters, resident in HBM before timing; each step
+moves 7.8 GB, far more than the 126 MB L2, so no L2 flush is needed.
+
+Printed: one JSON line (rank 0).  ``value`` is whole-job params/s over the K
+timed steps (CUDA events on the launching stream, max over ranks; N > 1 runs
+independent replicas, one per GPU, since the step itself has no exchange);
+``roofline`` reports the update kernel (the dominant one) against the measured
+HBM copy bandwidth; ``e2e`` times the same step through the public API with the
+gradients copied from pinned host memory every step; ``cpu_baseline`` times
+the CPU oracle (single thread) on a bounded leading slice of the workload.
+
+``--impl reference`` times the CPU oracle instead, on host cores, on bounded
+leading slices of the same workload (the oracle is the only reference
+implementation of this path).
+"""
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "params/sec and achieved HBM GB/s (fraction of B200 peak) per optimizer step"
+DEFAULT_WORKLOAD = "gpt2_medium"
+BYTES_UPDATE = 20        # per parameter: read g16 2 + w 4 + v 4, write w 4 + v 4 + w16 2
+BYTES_CHECK = 2          # per parameter: read g16
+READBACK_BYTES = 80      # the control block mpt_step copies back each step
+FALLBACK_HBM_GBS = 6650.0
+
+
+def parse_args():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["mpt", "reference"], default="mpt")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--e2e-steps", type=int, default=20)
+    ap.add_argument("--cpu-seconds", type=float, default=12.0,
+                    help="approximate CPU time spent timing the oracle baseline")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def measured_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def cpu_model():
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
+def host_cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region
+# ---------------------------------------------------------------------------
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.proc = None
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-i", str(gpu_index), "-lms", "50"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, ValueError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=10)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, smax, power, reasons = [], [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+                power.append(float(parts[3]))
+            except ValueError:
+                continue
+            for name, val in zip(names, parts[5:9]):
+                if val.lower() == "active":
+                    reasons.add(name)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        busy = [s for s, p in zip(sm, power) if p >= 0.5 * max(power)] or sm
+        return {"sm_mhz": statistics.median(busy), "sm_max_mhz": max(smax),
+                "reasons": sorted(reasons), "samples": len(sm),
+                "power_w_max": max(power)}
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle timing (baseline and the reference arm)
+# ---------------------------------------------------------------------------
+
+def oracle_sample(cfg, max_params, device):
+    """Inputs of a bounded leading slice of the workload, on the host."""
+    import numpy as np
+    import oracle
+    import workloads as W
+    from workloads.configs import truncated
+
+    sub = truncated(cfg, max_params)
+    layout = W.GradLayout(sub.sizes)
+    grads = W.make_grads(sub, 1, sub.scale0, layout, device).cpu()
+    hv = [v.numpy().view(np.uint16) for v in layout.views(grads)]
+    master = [m.cpu().numpy() for m in W.make_master(sub, device)]
+    return sub, hv, oracle.State.from_master(master)
+
+
+def time_oracle(cfg, sub, hv, state, steps):
+    import oracle
+    ocfg = oracle.scaler_cfg(backoff=cfg.backoff, growth=cfg.growth,
+                             growth_interval=cfg.growth_interval)
+    times = []
+    for _ in range(steps):
+        t0 = time.perf_counter()
+        oracle.step(state, hv, sub.scale0, cfg.lr, cfg.momentum, cfg.weight_decay,
+                    clip=cfg.clip, cfg=ocfg)
+        times.append(time.perf_counter() - t0)
+    return times
+
+
+def cpu_baseline(cfg, seconds, device):
+    # ~25-40 M params/s on one core: size the slice for a few steps of ~1/4 s each
+    sub, hv, state = oracle_sample(cfg, 8_000_000, device)
+    time_oracle(cfg, sub, hv, state, 1)                         # warm-up
+    per = statistics.median(time_oracle(cfg, sub, hv, state, 2))
+    steps = max(3, int(seconds / max(per, 1e-3)))
+    times = time_oracle(cfg, sub, hv, state, steps)
+    total = sum(times)
+    return {"value": sub.n_params * steps / total, "unit": "params/s", "cores": 1,
+            "kind": "oracle",
+            "sample": f"leading {sub.n_params} params of {cfg.name} ({len(sub.sizes)} tensors), "
+                      f"{steps} steps, single-threaded C oracle",
+            "host_cores": host_cores(), "cpu_model": cpu_model(), "seconds": total}
+
+
+def run_reference(args, cfg):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    import torch
+    device = "cuda" if torch.cuda.is_available() else "cpu"
+    sub, hv, state = oracle_sample(cfg, 4_000_000, device)
+    time_oracle(cfg, sub, hv, state, args.warmup)
+    times = time_oracle(cfg, sub, hv, state, args.steps)
+    total = sum(times)
+    value = sub.n_params * args.steps / total
+    sample = (f"each step: the leading {sub.n_params} params of {cfg.name} "
+              f"({len(sub.sizes)} tensors), single-threaded C oracle")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "params/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * total / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": {"workload": cfg.name, "params": cfg.n_params, "tensors": len(cfg.sizes),
+                   "sample_params": sub.n_params},
+        "cpu_baseline": {"value": value, "unit": "params/s", "cores": 1, "kind": "oracle",
+                         "sample": sample, "host_cores": host_cores(), "cpu_model": cpu_model()},
+        "e2e": {"value": value, "unit": "params/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------------------
+# the GPU arm
+# ---------------------------------------------------------------------------
+
+def run_mpt(args, cfg):
+    import torch
+    import torch.distributed as dist
+    import workloads as W
+    from loss_scaled_fp32_b200 import MPT, Config, grad_pointers
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    P = cfg.n_params
+    opt = MPT(cfg.sizes, Config(growth_interval=cfg.growth_interval), device=dev)
+    for i, m in enumerate(W.make_master(cfg, dev)):
+        opt.master(i).copy_(m)
+    opt.refresh_half()
+    layout = W.GradLayout(cfg.sizes)
+    sets = [W.make_grads(cfg, s, cfg.scale0, layout, dev) for s in (1, 2)]
+    ptrs = [grad_pointers(layout.views(g)) for g in sets]
+    S = cfg.scale0
+    stream = torch.cuda.current_stream(dev)
+    torch.cuda.synchronize(dev)
+
+    def step(k):
+        return opt.step(ptrs[k % 2], S, cfg.lr, cfg.momentum, cfg.weight_decay, cfg.clip,
+                        stream=stream)
+
+    for k in range(args.warmup):
+        step(k)
+    clocks = ClockSampler(local) if rank == 0 else None
+    time.sleep(0.3 if clocks else 0)                  # let nvidia-smi start sampling
+    opt.set_timing(True)
+    before = opt.stats()
+    barrier()
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    skipped = clipped = 0
+    for k in range(args.steps):
+        r = step(k)
+        skipped += r["found_inf"]
+        clipped += r["clipped"]
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    clock_info = clocks.stop() if clocks else None
+    opt.set_timing(False)
+    ms = e0.elapsed_time(e1)
+    after = opt.stats()
+    timed = after["timed_steps"] - before["timed_steps"]
+    check_ms = (after["check_ms_total"] - before["check_ms_total"]) / timed
+    update_ms = (after["update_ms_total"] - before["update_ms_total"]) / timed
+
+    ms_max = ms
+    if world > 1:
+        t = torch.tensor([ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_max = float(t.item())
+
+    # end to end through the public API: gradients from pinned host memory
+    # every step, result read back by the call itself
+    host = [torch.empty(g.numel(), dtype=torch.int16, pin_memory=True) for g in sets]
+    for h, g in zip(host, sets):
+        h.copy_(g)
+    torch.cuda.synchronize(dev)
+    dev_flat = sets[0]
+    barrier()
+    f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    f0.record(stream)
+    for k in range(args.e2e_steps):
+        dev_flat.copy_(host[k % 2], non_blocking=True)
+        opt.step(ptrs[0], S, cfg.lr, cfg.momentum, cfg.weight_decay, cfg.clip, stream=stream)
+    f1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = f0.elapsed_time(f1) / max(1, args.e2e_steps)
+    if world > 1:
+        t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+
+    base = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        base = cpu_baseline(cfg, args.cpu_seconds, dev)
+
+    if rank == 0:
+        peak, peak_kind = measured_peak()
+        ms_step = ms_max / args.steps
+        achieved_update = BYTES_UPDATE * P / (update_ms * 1e-3) / 1e9
+        achieved_check = BYTES_CHECK * P / (check_ms * 1e-3) / 1e9
+        traffic = load_traffic(cfg.name)
+        line = {
+            "metric": METRIC,
+            "value": world * P / (ms_step * 1e-3),
+            "unit": "params/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": ms_step,
+            "higher_is_better": True,
+            "scaling": "weak",
+            "vs_baseline": None,
+            "dtype": "f32",
+            "data": "synthetic (seeded FP16 gradients, random-init FP32 masters)",
+            "hbm_gbs": (BYTES_UPDATE + BYTES_CHECK) * P / (ms_step * 1e-3) / 1e9,
+            "hbm_frac_of_measured": (BYTES_UPDATE + BYTES_CHECK) * P / (ms_step * 1e-3) / 1e9 / peak,
+            "config": {"workload": cfg.name, "params": P, "tensors": len(cfg.sizes),
+                       "bytes_per_param": BYTES_UPDATE + BYTES_CHECK,
+                       "scale": S, "clip": cfg.clip, "lr": cfg.lr, "momentum": cfg.momentum,
+                       "weight_decay": cfg.weight_decay, "grad_sets": len(sets),
+                       "l2": "inputs larger than L2: 7.8 GB moved per step vs 126 MB L2",
+                       "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                       "clipped_steps": clipped, "skipped_steps": skipped},
+            "kernels_ms": {"check": check_ms, "update": update_ms,
+                           "host_and_readback": ms_step - check_ms - update_ms},
+            "roofline": {"kernel": "update_kernel", "bound": "hbm",
+                         "achieved": achieved_update, "peak": peak, "unit": "GB/s",
+                         "frac": achieved_update / peak, "peak_kind": peak_kind,
+                         "traffic": traffic,
+                         "algorithmic_bytes_per_launch": BYTES_UPDATE * P,
+                         "check_kernel": {"achieved": achieved_check,
+                                          "frac": achieved_check / peak,
+                                          "algorithmic_bytes_per_launch": BYTES_CHECK * P}},
+            "e2e": {"value": world * P / (e2e_ms * 1e-3), "unit": "params/s",
+                    "ms_per_step": e2e_ms,
+                    "h2d_bytes_per_step": sets[0].numel() * 2,
+                    "d2h_bytes_per_step": READBACK_BYTES},
+            "gpu_launches": 2 * args.steps,
+            "clocks": clock_info,
+            "cpu_baseline": base,
+        }
+        print(json.dumps(line), flush=True)
+    opt.close()
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+def load_traffic(workload):
+    """DRAM bytes per launch of the update kernel from the committed ncu
+    summary, if it was taken on the current kernel source; else None."""
+    try:
+        from loss_scaled_fp32_b200 import build as mbuild
+        path = os.path.join(ROOT, "profiles", "update_kernel_traffic.json")
+        with open(path) as f:
+            rec = json.load(f)
+        if rec.get("kernel_source_sha256") != mbuild.kernel_digest():
+            return None
+        return rec["dram_bytes_per_param"] * next(
+            c for c in [__import__("workloads").get(workload)]).n_params
+    except Exception:
+        return None
+
+
+def main():
+    args = parse_args()
+    import workloads as W
+    cfg = W.get(args.workload)
+    if args.impl == "reference":
+        return run_reference(args, cfg)
+    return run_mpt(args, cfg)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

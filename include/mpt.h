@@ -1,0 +1,185 @@
+/*
+ * mpt.h -- libmpt: the loss-scaled FP32-master SGD-momentum optimizer step of
+ * mixed-precision training, on one NVIDIA B200 (sm_100a).
+ *
+ * What one step computes (Micikevicius et al., "Mixed Precision Training",
+ * as explained by the paper-graph-ui.vercel.app analysis, section 3.4,
+ * "The Integrated Training Procedure (Figure 1)", Steps 5-7, and the
+ * azimuth.plus tutorial, "Loss scaling: why gradients vanish in FP16"):
+ *
+ *   given FP16 weight gradients g16 of a list of tensors, computed from a loss
+ *   multiplied by S, and per-parameter FP32 state (master w, momentum v):
+ *     1. found_inf = any g16 is +-inf or NaN, over the whole list   (Step 6)
+ *     2. g   = fp32(g16) * (1/S)                                     (Step 5)
+ *     3. norm = sqrt(sum g^2) over the whole list (binary64);
+ *        if clip > 0 and norm > clip: g = g * (clip / norm)  (global-L2 clip,
+ *        after unscaling: "Summary of Design Choices")
+ *     4. if found_inf: leave w, v and the FP16 copy untouched, S = S*beta
+ *                                                   (Step 6, Method 3)
+ *        else, per element, every operation rounded to binary32:
+ *          d = g + lambda*w        ("A subtle interaction: weight decay")
+ *          v = mu*v + d            (Step 7)
+ *          w = w - eta*v           (Step 7)
+ *          w16 = round_to_nearest_even_fp16(w)   (Step 1 of the next pass)
+ *     5. after N consecutive clean steps, S = S*alpha (dynamic scaling,
+ *        "Choosing the Loss Scaling Factor", Method 3)
+ *
+ * Conventions for every call:
+ *   - Every function returns an int status: MPT_OK (0) or a negative
+ *     MPT_ERR_* code.  No call aborts, throws, traps or prints.
+ *   - A handle is used by one host thread at a time.
+ *   - "device pointer" means memory of the CUDA device that is current when
+ *     mpt_create is called; every later call must run with that device current.
+ *   - cuda_stream arguments are cudaStream_t values passed as void*; NULL is
+ *     the legacy default stream.
+ *   - After MPT_ERR_CUDA the handle is broken: every later call except
+ *     mpt_stats, mpt_error_string and mpt_destroy returns MPT_ERR_BROKEN.
+ */
+#ifndef LIBMPT_MPT_H
+#define LIBMPT_MPT_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* ---- status codes ------------------------------------------------------- */
+#define MPT_OK 0
+#define MPT_ERR_INVALID_ARG (-1)  /* null or odd pointer, n <= 0, size <= 0,
+                                     S not finite or <= 0, lr / momentum /
+                                     weight decay / clip not finite          */
+#define MPT_ERR_WORKSPACE (-2)    /* workspace too small, not 256-B aligned,
+                                     or not device memory of this device    */
+#define MPT_ERR_CUDA (-3)         /* a CUDA runtime call failed             */
+#define MPT_ERR_DEVICE_CHECK (-4) /* checked mode found a work-table entry out
+                                     of bounds; that entry was not touched   */
+#define MPT_ERR_BROKEN (-5)       /* the handle saw MPT_ERR_CUDA earlier     */
+
+/* ---- configuration ------------------------------------------------------ */
+#define MPT_FLAG_CHECKED 0x1u     /* kernels validate every work-table entry
+                                     against the tensor sizes and arenas     */
+#define MPT_FLAG_COUNT_STALE 0x2u /* count elements whose master moved but
+                                     whose FP16 copy did not                 */
+
+typedef struct {
+    float backoff;            /* beta: S multiplier on overflow (default 0.5)      */
+    float growth;             /* alpha: S multiplier after N clean steps (2.0)     */
+    int32_t growth_interval;  /* N; 0 = constant S (an overflow still backs off) */
+    float min_scale;          /* lower bound of S after a backoff (2^-24)          */
+    float max_scale;          /* upper bound of S after a growth (2^24)            */
+    uint32_t flags;           /* MPT_FLAG_* (default 0)                            */
+    int32_t chunk_elems;      /* elements per work bin: a multiple of 2048 in
+                                 [2048, 2^20]; 0 = default (32768)                 */
+} mpt_config;
+
+/* ---- results ------------------------------------------------------------ */
+typedef struct {
+    int32_t found_inf;     /* 1: some gradient was +-inf/NaN; the update was
+                              skipped and the state is bitwise unchanged        */
+    int32_t clipped;       /* 1: clip > 0 and grad_norm > clip                  */
+    float new_scale;       /* S to use for the next step                        */
+    int32_t clean_run;     /* consecutive clean steps after this one            */
+    double grad_norm;      /* global L2 norm of the unscaled, unclipped
+                              gradients; +inf when found_inf                    */
+    float clip_coef;       /* clip / grad_norm when clipped, else 1             */
+    int32_t reserved;
+    uint64_t n_zero;       /* FP16 gradients equal to +-0                       */
+    uint64_t n_subnormal;  /* FP16 gradients with 0 < |g16| < 2^-14             */
+    uint64_t n_nonfinite;  /* FP16 gradients that are +-inf or NaN              */
+    uint64_t n_fp16_stale; /* MPT_FLAG_COUNT_STALE only, else 0: elements whose
+                              master changed while the rounded copy did not     */
+} mpt_step_result;
+
+typedef struct {
+    uint64_t steps;           /* mpt_step calls that completed                  */
+    uint64_t skipped;         /* of which were skipped on overflow              */
+    float scale;              /* current S (last new_scale, or the value set)   */
+    int32_t clean_run;        /* current clean-step counter                     */
+    mpt_step_result last;     /* result of the last completed step              */
+    uint64_t n_fp16_stale_total;
+    uint64_t timed_steps;     /* steps timed while mpt_set_timing was on        */
+    double check_ms_total;    /* summed CUDA-event durations of the check       */
+    double update_ms_total;   /* kernel and of the update kernel over them      */
+} mpt_stats_t;
+
+typedef struct mpt_handle mpt_handle;  /* opaque */
+
+/* ---- calls -------------------------------------------------------------- */
+
+/* Fill *cfg with the defaults listed in mpt_config.
+ * Errors: MPT_ERR_INVALID_ARG (cfg NULL). */
+int mpt_config_init(mpt_config* cfg);
+
+/* Bytes of device workspace mpt_create needs for n tensors with the given
+ * element counts (host array sizes[n]); cfg NULL = defaults.  The workspace
+ * holds the FP32 master arena, the FP32 momentum arena and the FP16
+ * working-copy arena (each tensor at a 16-element-aligned offset) plus the
+ * work tables and a small control block.
+ * Errors: MPT_ERR_INVALID_ARG (a pointer NULL, n <= 0, a size <= 0, bad cfg). */
+int mpt_workspace_bytes(const int64_t* sizes, int32_t n, const mpt_config* cfg,
+                        size_t* bytes);
+
+/* Create a handle over a caller-owned device workspace d_workspace of
+ * ws_bytes bytes (256-byte aligned, at least mpt_workspace_bytes).  Builds and
+ * uploads the work tables and zeroes the three arenas and the control block,
+ * synchronously.  The caller then writes the initial master weights through
+ * mpt_tensor_views and calls mpt_refresh_half.  The workspace and the
+ * gradient buffers belong to the caller and must outlive the handle; the
+ * library owns only host tables and two small pinned host buffers.  The loss
+ * scale starts at 1 with a clean-step counter of 0 (mpt_set_scaler_state).
+ * Errors: MPT_ERR_INVALID_ARG, MPT_ERR_WORKSPACE, MPT_ERR_CUDA. */
+int mpt_create(const int64_t* sizes, int32_t n, const mpt_config* cfg,
+               void* d_workspace, size_t ws_bytes, mpt_handle** out);
+
+/* Device pointers to tensor i's slices of the arenas: FP32 master, FP32
+ * momentum and FP16 working copy (binary16, sizes[i] elements each, 64-byte
+ * aligned).  Any output pointer may be NULL.
+ * Errors: MPT_ERR_INVALID_ARG (h NULL, i out of range). */
+int mpt_tensor_views(const mpt_handle* h, int32_t i, float** master,
+                     float** momentum, void** w16_half);
+
+/* Rewrite every FP16 working copy from its FP32 master: w16 = RNE_fp16(w)
+ * (Step 1 of the training iteration).  Asynchronous on cuda_stream.
+ * Errors: MPT_ERR_INVALID_ARG, MPT_ERR_CUDA, MPT_ERR_BROKEN. */
+int mpt_refresh_half(mpt_handle* h, void* cuda_stream);
+
+/* One optimizer step.  d_grads_half is a HOST array of n DEVICE pointers, the
+ * FP16 (binary16) gradients of the n tensors, computed from a loss multiplied
+ * by `scale` (any 2-byte alignment; contents are only read).  lr, momentum
+ * and weight_decay are eta, mu and lambda; clip <= 0 disables clipping.
+ * Work is queued on cuda_stream and the call waits for it (it reads the
+ * result back), then updates the handle's scale state: out->new_scale is
+ * the S to pass to the next step.  On overflow the arenas are untouched.
+ * Errors: MPT_ERR_INVALID_ARG, MPT_ERR_CUDA, MPT_ERR_DEVICE_CHECK,
+ * MPT_ERR_BROKEN; on any error *out is not written and the scale state does
+ * not change. */
+int mpt_step(mpt_handle* h, const void* const* d_grads_half, float scale,
+             float lr, float momentum, float weight_decay, float clip,
+             void* cuda_stream, mpt_step_result* out);
+
+/* Counters and the last result.  Errors: MPT_ERR_INVALID_ARG. */
+int mpt_stats(const mpt_handle* h, mpt_stats_t* out);
+
+/* Read / set the loss-scale state (checkpoint and resume).  set requires a
+ * finite scale > 0 and clean_run >= 0.  Errors: MPT_ERR_INVALID_ARG. */
+int mpt_get_scaler_state(const mpt_handle* h, float* scale, int32_t* clean_run);
+int mpt_set_scaler_state(mpt_handle* h, float scale, int32_t clean_run);
+
+/* Time both kernels of every following step with CUDA events recorded on the
+ * step's stream (summed into mpt_stats_t); enable = 0 turns it off.
+ * Errors: MPT_ERR_INVALID_ARG, MPT_ERR_CUDA. */
+int mpt_set_timing(mpt_handle* h, int32_t enable);
+
+/* Release the handle's host resources.  The workspace is the caller's and is
+ * not freed.  NULL is accepted. */
+int mpt_destroy(mpt_handle* h);
+
+/* Static description of a status code (never NULL). */
+const char* mpt_error_string(int code);
+
+#ifdef __cplusplus
+}
+#endif
+#endif

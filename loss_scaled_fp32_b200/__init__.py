@@ -1,0 +1,234 @@
+"""Python binding of libmpt: the loss-scaled FP32-master optimizer step on B200.
+
+Argument marshalling only (ctypes over the C ABI in ``include/mpt.h``): every
+step of the path runs in the library's CUDA kernels.  PyTorch supplies the
+device workspace and the stream.  There is no CPU fallback: if ``libmpt.so``
+cannot be loaded (or built with nvcc), importing the library fails loudly.
+
+    opt = MPT(sizes, Config(growth_interval=4))
+    for i, w in enumerate(initial_weights):
+        opt.master(i).copy_(w)
+    opt.refresh_half()
+    opt.set_scaler_state(2.0 ** 16)
+    res = opt.step(grads, scale=opt.scale, lr=0.01, momentum=0.9,
+                   weight_decay=1e-4, clip=1.0)
+"""
+import ctypes
+import os
+
+from . import build as _build
+
+__all__ = ["MPT", "Config", "MptError", "lib", "grad_pointers",
+           "MPT_FLAG_CHECKED", "MPT_FLAG_COUNT_STALE"]
+
+MPT_FLAG_CHECKED = 0x1
+MPT_FLAG_COUNT_STALE = 0x2
+
+MPT_OK = 0
+MPT_ERR_INVALID_ARG = -1
+MPT_ERR_WORKSPACE = -2
+MPT_ERR_CUDA = -3
+MPT_ERR_DEVICE_CHECK = -4
+MPT_ERR_BROKEN = -5
+
+
+class MptError(RuntimeError):
+    def __init__(self, code, what):
+        self.code = code
+        super().__init__(f"{what}: {lib().mpt_error_string(code).decode()} ({code})")
+
+
+class Config(ctypes.Structure):
+    _fields_ = [("backoff", ctypes.c_float), ("growth", ctypes.c_float),
+                ("growth_interval", ctypes.c_int32), ("min_scale", ctypes.c_float),
+                ("max_scale", ctypes.c_float), ("flags", ctypes.c_uint32),
+                ("chunk_elems", ctypes.c_int32)]
+
+    def __init__(self, **kw):
+        super().__init__()
+        lib().mpt_config_init(ctypes.byref(self))
+        for k, v in kw.items():
+            if k not in dict(self._fields_):
+                raise TypeError(f"unknown config field {k}")
+            setattr(self, k, v)
+
+
+class StepResult(ctypes.Structure):
+    _fields_ = [("found_inf", ctypes.c_int32), ("clipped", ctypes.c_int32),
+                ("new_scale", ctypes.c_float), ("clean_run", ctypes.c_int32),
+                ("grad_norm", ctypes.c_double), ("clip_coef", ctypes.c_float),
+                ("reserved", ctypes.c_int32), ("n_zero", ctypes.c_uint64),
+                ("n_subnormal", ctypes.c_uint64), ("n_nonfinite", ctypes.c_uint64),
+                ("n_fp16_stale", ctypes.c_uint64)]
+
+    def as_dict(self):
+        return {k: getattr(self, k) for k, _ in self._fields_ if k != "reserved"}
+
+
+class Stats(ctypes.Structure):
+    _fields_ = [("steps", ctypes.c_uint64), ("skipped", ctypes.c_uint64),
+                ("scale", ctypes.c_float), ("clean_run", ctypes.c_int32),
+                ("last", StepResult), ("n_fp16_stale_total", ctypes.c_uint64),
+                ("timed_steps", ctypes.c_uint64), ("check_ms_total", ctypes.c_double),
+                ("update_ms_total", ctypes.c_double)]
+
+    def as_dict(self):
+        d = {k: getattr(self, k) for k, _ in self._fields_}
+        d["last"] = self.last.as_dict()
+        return d
+
+
+_LIB = None
+
+
+def lib():
+    """Load (building with nvcc if needed) ``libmpt.so``; raises if impossible."""
+    global _LIB
+    if _LIB is None:
+        path = _build.LIB
+        if not os.path.exists(path) or os.environ.get("MPT_REBUILD"):
+            path = _build.build()
+        L = ctypes.CDLL(path)
+        vp, i32, f32 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_float
+        sig = {
+            "mpt_config_init": [ctypes.POINTER(Config)],
+            "mpt_workspace_bytes": [vp, i32, ctypes.POINTER(Config), ctypes.POINTER(ctypes.c_size_t)],
+            "mpt_create": [vp, i32, ctypes.POINTER(Config), vp, ctypes.c_size_t, ctypes.POINTER(vp)],
+            "mpt_tensor_views": [vp, i32, ctypes.POINTER(vp), ctypes.POINTER(vp), ctypes.POINTER(vp)],
+            "mpt_refresh_half": [vp, vp],
+            "mpt_step": [vp, vp, f32, f32, f32, f32, f32, vp, ctypes.POINTER(StepResult)],
+            "mpt_stats": [vp, ctypes.POINTER(Stats)],
+            "mpt_get_scaler_state": [vp, ctypes.POINTER(f32), ctypes.POINTER(i32)],
+            "mpt_set_scaler_state": [vp, f32, i32],
+            "mpt_set_timing": [vp, i32],
+            "mpt_destroy": [vp],
+        }
+        for name, args in sig.items():
+            fn = getattr(L, name)
+            fn.argtypes = args
+            fn.restype = ctypes.c_int
+        L.mpt_error_string.argtypes = [ctypes.c_int]
+        L.mpt_error_string.restype = ctypes.c_char_p
+        _LIB = L
+    return _LIB
+
+
+def _check(code, what):
+    if code != MPT_OK:
+        raise MptError(code, what)
+
+
+def grad_pointers(tensors):
+    """Host array of device pointers (build once, reuse across steps)."""
+    return (ctypes.c_void_p * len(tensors))(*[t.data_ptr() for t in tensors])
+
+
+def _stream_ptr(stream, device):
+    import torch
+    s = stream if stream is not None else torch.cuda.current_stream(device)
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+class MPT:
+    """One optimizer over a fixed list of tensor sizes (one CUDA device)."""
+
+    def __init__(self, sizes, config=None, device=None):
+        import torch
+        self.sizes = [int(s) for s in sizes]
+        self.n = len(self.sizes)
+        self.config = config if config is not None else Config()
+        self.device = torch.device(device if device is not None else "cuda", )
+        if self.device.index is None:
+            self.device = torch.device("cuda", torch.cuda.current_device())
+        self._sizes_c = (ctypes.c_int64 * self.n)(*self.sizes)
+        nbytes = ctypes.c_size_t()
+        _check(lib().mpt_workspace_bytes(self._sizes_c, self.n, ctypes.byref(self.config),
+                                         ctypes.byref(nbytes)), "mpt_workspace_bytes")
+        self.workspace_bytes = nbytes.value
+        self.workspace = torch.empty(self.workspace_bytes, dtype=torch.uint8, device=self.device)
+        h = ctypes.c_void_p()
+        with torch.cuda.device(self.device):
+            _check(lib().mpt_create(self._sizes_c, self.n, ctypes.byref(self.config),
+                                    ctypes.c_void_p(self.workspace.data_ptr()),
+                                    self.workspace_bytes, ctypes.byref(h)), "mpt_create")
+        self._h = h
+        self._views = [self._make_views(i) for i in range(self.n)]
+        self._ptr_cache = None
+
+    # -- state views ---------------------------------------------------------
+    def _make_views(self, i):
+        import torch
+        m, v, w = ctypes.c_void_p(), ctypes.c_void_p(), ctypes.c_void_p()
+        _check(lib().mpt_tensor_views(self._h, i, ctypes.byref(m), ctypes.byref(v),
+                                      ctypes.byref(w)), "mpt_tensor_views")
+        base = self.workspace.data_ptr()
+        n = self.sizes[i]
+        ws = self.workspace
+        return (ws[m.value - base: m.value - base + 4 * n].view(torch.float32),
+                ws[v.value - base: v.value - base + 4 * n].view(torch.float32),
+                ws[w.value - base: w.value - base + 2 * n].view(torch.float16))
+
+    def master(self, i):
+        return self._views[i][0]
+
+    def momentum(self, i):
+        return self._views[i][1]
+
+    def w16(self, i):
+        return self._views[i][2]
+
+    # -- calls ---------------------------------------------------------------
+    def refresh_half(self, stream=None):
+        _check(lib().mpt_refresh_half(self._h, _stream_ptr(stream, self.device)),
+               "mpt_refresh_half")
+
+    def step(self, grads, scale, lr, momentum, weight_decay, clip=0.0, stream=None):
+        """``grads``: list of FP16 (or int16 bit-pattern) CUDA tensors, or an
+        array from :func:`grad_pointers`.  Returns the step result as a dict."""
+        if isinstance(grads, ctypes.Array):
+            ptrs = grads
+        else:
+            if len(grads) != self.n:
+                raise ValueError(f"expected {self.n} gradient tensors, got {len(grads)}")
+            for g, n in zip(grads, self.sizes):
+                if g.numel() != n or g.element_size() != 2 or g.device != self.device:
+                    raise ValueError("gradient tensor does not match its size/dtype/device")
+                if not g.is_contiguous():
+                    raise ValueError("gradient tensors must be contiguous")
+            ptrs = grad_pointers(grads)
+        r = StepResult()
+        _check(lib().mpt_step(self._h, ptrs, scale, lr, momentum, weight_decay, clip,
+                              _stream_ptr(stream, self.device), ctypes.byref(r)), "mpt_step")
+        return r.as_dict()
+
+    def stats(self):
+        s = Stats()
+        _check(lib().mpt_stats(self._h, ctypes.byref(s)), "mpt_stats")
+        return s.as_dict()
+
+    @property
+    def scale(self):
+        return self.scaler_state()[0]
+
+    def scaler_state(self):
+        s, c = ctypes.c_float(), ctypes.c_int32()
+        _check(lib().mpt_get_scaler_state(self._h, ctypes.byref(s), ctypes.byref(c)),
+               "mpt_get_scaler_state")
+        return s.value, c.value
+
+    def set_scaler_state(self, scale, clean_run=0):
+        _check(lib().mpt_set_scaler_state(self._h, scale, clean_run), "mpt_set_scaler_state")
+
+    def set_timing(self, enable=True):
+        _check(lib().mpt_set_timing(self._h, 1 if enable else 0), "mpt_set_timing")
+
+    def close(self):
+        if getattr(self, "_h", None):
+            lib().mpt_destroy(self._h)
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass

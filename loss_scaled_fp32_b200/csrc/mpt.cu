@@ -1,0 +1,554 @@
+// mpt.cu -- host side of libmpt: the C ABI declared in include/mpt.h.
+//
+// One step = two kernel launches on the caller's stream and one 80-byte
+// read-back of the control block:
+//   check_kernel  (2 B/param)  overflow flag, range counts, sum of squares,
+//                              last-CTA finish -> norm, clip coefficient
+//   update_kernel (20 B/param) fused unscale/clip/decay/momentum/master/FP16,
+//                              or counting only when the step overflowed
+// The launch order alone carries the check result to the update, so no host
+// decision sits between the two kernels.  The loss-scale state machine runs on
+// the host once the result is back.
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdlib>
+#include <cstring>
+#include <new>
+#include <vector>
+
+#include "../../include/mpt.h"
+#include "mpt_internal.h"
+#include "mpt_kernels.cuh"
+
+using namespace mpt;
+
+static_assert(sizeof(Ctrl) == 80, "the control block read back each step is 80 bytes");
+
+namespace {
+
+constexpr size_t kRegionAlign = 256;
+
+size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+struct Layout {
+    std::vector<int64_t> arena_off;
+    int64_t arena_total = 0;
+    std::vector<Bin> bins;
+    std::vector<Seg> segs;
+    size_t off_ctrl = 0, off_partials = 0, off_ptrs = 0, off_tinfo = 0, off_bins = 0,
+           off_segs = 0, off_master = 0, off_momentum = 0, off_w16 = 0, total = 0;
+};
+
+bool config_ok(const mpt_config& c)
+{
+    if (!(c.backoff > 0.0f && c.backoff <= 1.0f) || !(c.growth >= 1.0f) || !std::isfinite(c.growth))
+        return false;
+    if (c.growth_interval < 0)
+        return false;
+    if (!(c.min_scale > 0.0f) || !std::isfinite(c.max_scale) || !(c.max_scale >= c.min_scale))
+        return false;
+    if (c.flags & ~(MPT_FLAG_CHECKED | MPT_FLAG_COUNT_STALE))
+        return false;
+    if (c.chunk_elems != 0 && (c.chunk_elems < kChunkQuantum || c.chunk_elems > kMaxChunk ||
+                               c.chunk_elems % kChunkQuantum != 0))
+        return false;
+    return true;
+}
+
+mpt_config defaults()
+{
+    mpt_config c;
+    c.backoff = 0.5f;
+    c.growth = 2.0f;
+    c.growth_interval = 0;
+    c.min_scale = std::ldexp(1.0f, -24);
+    c.max_scale = std::ldexp(1.0f, 24);
+    c.flags = 0;
+    c.chunk_elems = 0;
+    return c;
+}
+
+// Arena offsets (16-element aligned) and the work bins: every tensor larger
+// than kSmallTensor is cut into chunk-sized ranges, one bin each; the small
+// tensors are packed, in list order, into bins of at most `chunk` elements.
+int build_layout(const int64_t* sizes, int32_t n, int32_t chunk, Layout& L)
+{
+    L.arena_off.resize(n);
+    int64_t off = 0;
+    for (int32_t i = 0; i < n; ++i) {
+        if (sizes[i] <= 0)
+            return MPT_ERR_INVALID_ARG;
+        L.arena_off[i] = off;
+        off += (sizes[i] + kArenaAlign - 1) / kArenaAlign * kArenaAlign;
+    }
+    L.arena_total = off;
+
+    for (int32_t i = 0; i < n; ++i) {
+        if (sizes[i] <= kSmallTensor)
+            continue;
+        for (int64_t c = 0; c < sizes[i]; c += chunk) {
+            Seg s{};
+            s.tensor_begin = c;
+            s.arena_begin = L.arena_off[i] + c;
+            s.tensor = i;
+            s.len = (int32_t)std::min<int64_t>(chunk, sizes[i] - c);
+            s.local_begin = 0;
+            Bin b{};
+            b.first_seg = (int32_t)L.segs.size();
+            b.n_segs = 1;
+            b.n_elems = s.len;
+            b.kind = kChunkBin;
+            L.segs.push_back(s);
+            L.bins.push_back(b);
+        }
+    }
+    Bin open{};
+    bool have_open = false;
+    for (int32_t i = 0; i < n; ++i) {
+        if (sizes[i] > kSmallTensor)
+            continue;
+        const int32_t len = (int32_t)sizes[i];
+        if (have_open && (open.n_elems + len > chunk || open.n_segs == kMaxPackedSegs)) {
+            L.bins.push_back(open);
+            have_open = false;
+        }
+        if (!have_open) {
+            open = Bin{};
+            open.first_seg = (int32_t)L.segs.size();
+            open.kind = kPackedBin;
+            have_open = true;
+        }
+        Seg s{};
+        s.tensor_begin = 0;
+        s.arena_begin = L.arena_off[i];
+        s.tensor = i;
+        s.len = len;
+        s.local_begin = open.n_elems;
+        L.segs.push_back(s);
+        open.n_segs += 1;
+        open.n_elems += len;
+    }
+    if (have_open)
+        L.bins.push_back(open);
+    if (L.bins.size() > 0x7fffffffu || L.segs.size() > 0x7fffffffu)
+        return MPT_ERR_INVALID_ARG;
+
+    size_t p = 0;
+    auto region = [&](size_t bytes) {
+        const size_t at = p;
+        p = round_up(p + bytes, kRegionAlign);
+        return at;
+    };
+    L.off_ctrl = region(sizeof(Ctrl));
+    L.off_partials = region(sizeof(double) * L.bins.size());
+    L.off_ptrs = region(sizeof(void*) * (size_t)n);
+    L.off_tinfo = region(sizeof(TensorInfo) * (size_t)n);
+    L.off_bins = region(sizeof(Bin) * L.bins.size());
+    L.off_segs = region(sizeof(Seg) * L.segs.size());
+    L.off_master = region(sizeof(float) * (size_t)L.arena_total);
+    L.off_momentum = region(sizeof(float) * (size_t)L.arena_total);
+    L.off_w16 = region(sizeof(uint16_t) * (size_t)L.arena_total);
+    L.total = p;
+    return MPT_OK;
+}
+
+bool finite(float x) { return std::isfinite(x); }
+
+}  // namespace
+
+struct mpt_handle {
+    int device = 0;
+    int32_t n = 0;
+    mpt_config cfg{};
+    Layout L;
+    char* ws = nullptr;
+    // device views into the workspace
+    Ctrl* d_ctrl = nullptr;
+    double* d_partials = nullptr;
+    const uint16_t** d_ptrs = nullptr;
+    TensorInfo* d_tinfo = nullptr;
+    Bin* d_bins = nullptr;
+    Seg* d_segs = nullptr;
+    float* d_master = nullptr;
+    float* d_momentum = nullptr;
+    uint16_t* d_w16 = nullptr;
+    // host state
+    std::vector<const void*> last_ptrs;
+    bool ptrs_uploaded = false;
+    const void** pinned_ptrs = nullptr;  // staging of the pointer table
+    Ctrl* mailbox = nullptr;             // pinned copy of the control block
+    float scale = 1.0f;
+    int32_t clean_run = 0;
+    mpt_stats_t stats{};
+    bool broken = false;
+    bool timing = false;
+    cudaEvent_t ev[3] = {nullptr, nullptr, nullptr};
+};
+
+static void release(mpt_handle* h)
+{
+    if (!h)
+        return;
+    for (cudaEvent_t& e : h->ev)
+        if (e)
+            cudaEventDestroy(e);
+    if (h->pinned_ptrs)
+        cudaFreeHost(h->pinned_ptrs);
+    if (h->mailbox)
+        cudaFreeHost(h->mailbox);
+    delete h;
+}
+
+// Loss-scale state machine (dynamic loss scaling): back off on overflow,
+// grow after growth_interval consecutive clean steps.
+static float next_scale(const mpt_config& c, bool found_inf, float scale, int32_t& clean)
+{
+    if (found_inf) {
+        clean = 0;
+        const float s = scale * c.backoff;
+        return s < c.min_scale ? c.min_scale : s;
+    }
+    clean += 1;
+    if (c.growth_interval > 0 && clean >= c.growth_interval) {
+        clean = 0;
+        const float s = scale * c.growth;
+        return s > c.max_scale ? c.max_scale : s;
+    }
+    return scale;
+}
+
+template <bool kPow2, bool kChecked>
+static void launch_check(const CheckArgs& a, cudaStream_t st)
+{
+    check_kernel<kPow2, kChecked><<<a.t.nbins, kThreads, 0, st>>>(a);
+}
+
+template <bool kStale, bool kChecked>
+static void launch_update(const UpdateArgs& a, cudaStream_t st)
+{
+    update_kernel<kStale, kChecked><<<a.t.nbins, kThreads, 0, st>>>(a);
+}
+
+extern "C" {
+
+int mpt_config_init(mpt_config* cfg)
+{
+    if (!cfg)
+        return MPT_ERR_INVALID_ARG;
+    *cfg = defaults();
+    return MPT_OK;
+}
+
+int mpt_workspace_bytes(const int64_t* sizes, int32_t n, const mpt_config* cfg, size_t* bytes)
+{
+    if (!sizes || !bytes || n <= 0)
+        return MPT_ERR_INVALID_ARG;
+    const mpt_config c = cfg ? *cfg : defaults();
+    if (!config_ok(c))
+        return MPT_ERR_INVALID_ARG;
+    Layout L;
+    const int rc = build_layout(sizes, n, c.chunk_elems ? c.chunk_elems : kDefaultChunk, L);
+    if (rc != MPT_OK)
+        return rc;
+    *bytes = L.total;
+    return MPT_OK;
+}
+
+int mpt_create(const int64_t* sizes, int32_t n, const mpt_config* cfg, void* d_workspace,
+               size_t ws_bytes, mpt_handle** out)
+{
+    if (!sizes || n <= 0 || !out)
+        return MPT_ERR_INVALID_ARG;
+    *out = nullptr;
+    const mpt_config c = cfg ? *cfg : defaults();
+    if (!config_ok(c))
+        return MPT_ERR_INVALID_ARG;
+    mpt_handle* h = new (std::nothrow) mpt_handle();
+    if (!h)
+        return MPT_ERR_INVALID_ARG;
+    h->cfg = c;
+    h->n = n;
+    int rc = build_layout(sizes, n, c.chunk_elems ? c.chunk_elems : kDefaultChunk, h->L);
+    if (rc != MPT_OK) {
+        release(h);
+        return rc;
+    }
+    if (!d_workspace || (reinterpret_cast<uintptr_t>(d_workspace) % kRegionAlign) != 0 ||
+        ws_bytes < h->L.total) {
+        release(h);
+        return MPT_ERR_WORKSPACE;
+    }
+    if (cudaGetDevice(&h->device) != cudaSuccess) {
+        release(h);
+        return MPT_ERR_CUDA;
+    }
+    cudaPointerAttributes attr;
+    if (cudaPointerGetAttributes(&attr, d_workspace) != cudaSuccess ||
+        attr.type != cudaMemoryTypeDevice || attr.device != h->device) {
+        cudaGetLastError();
+        release(h);
+        return MPT_ERR_WORKSPACE;
+    }
+
+    char* ws = static_cast<char*>(d_workspace);
+    const Layout& L = h->L;
+    h->ws = ws;
+    h->d_ctrl = reinterpret_cast<Ctrl*>(ws + L.off_ctrl);
+    h->d_partials = reinterpret_cast<double*>(ws + L.off_partials);
+    h->d_ptrs = reinterpret_cast<const uint16_t**>(ws + L.off_ptrs);
+    h->d_tinfo = reinterpret_cast<TensorInfo*>(ws + L.off_tinfo);
+    h->d_bins = reinterpret_cast<Bin*>(ws + L.off_bins);
+    h->d_segs = reinterpret_cast<Seg*>(ws + L.off_segs);
+    h->d_master = reinterpret_cast<float*>(ws + L.off_master);
+    h->d_momentum = reinterpret_cast<float*>(ws + L.off_momentum);
+    h->d_w16 = reinterpret_cast<uint16_t*>(ws + L.off_w16);
+
+    std::vector<TensorInfo> tinfo(n);
+    for (int32_t i = 0; i < n; ++i) {
+        tinfo[i].size = sizes[i];
+        tinfo[i].arena_off = L.arena_off[i];
+    }
+    bool ok = cudaMemcpy(h->d_tinfo, tinfo.data(), sizeof(TensorInfo) * n, cudaMemcpyHostToDevice) == cudaSuccess &&
+              cudaMemcpy(h->d_bins, L.bins.data(), sizeof(Bin) * L.bins.size(), cudaMemcpyHostToDevice) == cudaSuccess &&
+              cudaMemcpy(h->d_segs, L.segs.data(), sizeof(Seg) * L.segs.size(), cudaMemcpyHostToDevice) == cudaSuccess &&
+              cudaMemset(h->d_ctrl, 0, sizeof(Ctrl)) == cudaSuccess &&
+              cudaMemset(h->d_ptrs, 0, sizeof(void*) * n) == cudaSuccess &&
+              cudaMemset(ws + L.off_master, 0, L.total - L.off_master) == cudaSuccess &&
+              cudaHostAlloc(reinterpret_cast<void**>(&h->pinned_ptrs), sizeof(void*) * n, cudaHostAllocDefault) == cudaSuccess &&
+              cudaHostAlloc(reinterpret_cast<void**>(&h->mailbox), sizeof(Ctrl), cudaHostAllocDefault) == cudaSuccess &&
+              cudaDeviceSynchronize() == cudaSuccess;
+    if (!ok) {
+        cudaGetLastError();
+        release(h);
+        return MPT_ERR_CUDA;
+    }
+    h->last_ptrs.assign(n, nullptr);
+    h->stats.scale = h->scale;
+    *out = h;
+    return MPT_OK;
+}
+
+int mpt_tensor_views(const mpt_handle* h, int32_t i, float** master, float** momentum,
+                     void** w16_half)
+{
+    if (!h || i < 0 || i >= h->n)
+        return MPT_ERR_INVALID_ARG;
+    const int64_t off = h->L.arena_off[i];
+    if (master)
+        *master = h->d_master + off;
+    if (momentum)
+        *momentum = h->d_momentum + off;
+    if (w16_half)
+        *w16_half = h->d_w16 + off;
+    return MPT_OK;
+}
+
+int mpt_refresh_half(mpt_handle* h, void* cuda_stream)
+{
+    if (!h)
+        return MPT_ERR_INVALID_ARG;
+    if (h->broken)
+        return MPT_ERR_BROKEN;
+    const int64_t n4 = h->L.arena_total / 4;
+    const int64_t want = (n4 + kThreads - 1) / kThreads;
+    const int blocks = (int)std::max<int64_t>(1, std::min<int64_t>(want, 148 * 16));
+    refresh_kernel<<<blocks, kThreads, 0, static_cast<cudaStream_t>(cuda_stream)>>>(
+        reinterpret_cast<const float4*>(h->d_master), reinterpret_cast<uint2*>(h->d_w16), n4);
+    if (cudaGetLastError() != cudaSuccess) {
+        h->broken = true;
+        return MPT_ERR_CUDA;
+    }
+    return MPT_OK;
+}
+
+int mpt_step(mpt_handle* h, const void* const* d_grads_half, float scale, float lr, float momentum,
+             float weight_decay, float clip, void* cuda_stream, mpt_step_result* out)
+{
+    if (!h || !d_grads_half || !out)
+        return MPT_ERR_INVALID_ARG;
+    if (h->broken)
+        return MPT_ERR_BROKEN;
+    if (!finite(scale) || !(scale > 0.0f) || !finite(lr) || !finite(momentum) ||
+        !finite(weight_decay) || !finite(clip))
+        return MPT_ERR_INVALID_ARG;
+    for (int32_t i = 0; i < h->n; ++i) {
+        const uintptr_t p = reinterpret_cast<uintptr_t>(d_grads_half[i]);
+        if (p == 0 || (p & 1))
+            return MPT_ERR_INVALID_ARG;
+    }
+    cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
+    const size_t ptr_bytes = sizeof(void*) * (size_t)h->n;
+
+    // The pointer table crosses to the device only when it changed.
+    if (!h->ptrs_uploaded || std::memcmp(h->last_ptrs.data(), d_grads_half, ptr_bytes) != 0) {
+        std::memcpy(h->pinned_ptrs, d_grads_half, ptr_bytes);
+        if (cudaMemcpyAsync(h->d_ptrs, h->pinned_ptrs, ptr_bytes, cudaMemcpyHostToDevice, st) != cudaSuccess) {
+            h->broken = true;
+            return MPT_ERR_CUDA;
+        }
+        std::memcpy(h->last_ptrs.data(), d_grads_half, ptr_bytes);
+        h->ptrs_uploaded = true;
+    }
+
+    Tables t;
+    t.bins = h->d_bins;
+    t.segs = h->d_segs;
+    t.tensors = h->d_tinfo;
+    t.grads = h->d_ptrs;
+    t.nbins = (int32_t)h->L.bins.size();
+    t.nsegs = (int32_t)h->L.segs.size();
+    t.ntensors = h->n;
+    t.pad = 0;
+    t.arena_total = h->L.arena_total;
+
+    CheckArgs ca;
+    ca.t = t;
+    ca.partials = h->d_partials;
+    ca.ctrl = h->d_ctrl;
+    ca.inv_scale = 1.0f / scale;
+    ca.clip = clip;
+    int e2 = 0;
+    const bool pow2 = std::frexp(scale, &e2) == 0.5f && (e2 - 1) >= -15 && (e2 - 1) <= 100;
+    ca.dscale = pow2 ? std::ldexp(1.0, 1008 - (e2 - 1)) : 0.0;
+
+    UpdateArgs ua;
+    ua.t = t;
+    ua.master = h->d_master;
+    ua.momentum = h->d_momentum;
+    ua.w16 = h->d_w16;
+    ua.ctrl = h->d_ctrl;
+    ua.inv_scale = ca.inv_scale;
+    ua.lr = lr;
+    ua.mu = momentum;
+    ua.wd = weight_decay;
+
+    const bool checked = (h->cfg.flags & MPT_FLAG_CHECKED) != 0;
+    const bool stale = (h->cfg.flags & MPT_FLAG_COUNT_STALE) != 0;
+    bool ok = true;
+    if (h->timing)
+        ok = ok && cudaEventRecord(h->ev[0], st) == cudaSuccess;
+    if (pow2)
+        checked ? launch_check<true, true>(ca, st) : launch_check<true, false>(ca, st);
+    else
+        checked ? launch_check<false, true>(ca, st) : launch_check<false, false>(ca, st);
+    if (h->timing)
+        ok = ok && cudaEventRecord(h->ev[1], st) == cudaSuccess;
+    if (stale)
+        checked ? launch_update<true, true>(ua, st) : launch_update<true, false>(ua, st);
+    else
+        checked ? launch_update<false, true>(ua, st) : launch_update<false, false>(ua, st);
+    if (h->timing)
+        ok = ok && cudaEventRecord(h->ev[2], st) == cudaSuccess;
+    ok = ok && cudaGetLastError() == cudaSuccess;
+    ok = ok && cudaMemcpyAsync(h->mailbox, h->d_ctrl, sizeof(Ctrl), cudaMemcpyDeviceToHost, st) == cudaSuccess;
+    ok = ok && cudaStreamSynchronize(st) == cudaSuccess;
+    if (!ok) {
+        cudaGetLastError();
+        h->broken = true;
+        h->ptrs_uploaded = false;
+        return MPT_ERR_CUDA;
+    }
+    if (h->timing) {
+        float t01 = 0.0f, t12 = 0.0f;
+        if (cudaEventElapsedTime(&t01, h->ev[0], h->ev[1]) == cudaSuccess &&
+            cudaEventElapsedTime(&t12, h->ev[1], h->ev[2]) == cudaSuccess) {
+            h->stats.check_ms_total += t01;
+            h->stats.update_ms_total += t12;
+            h->stats.timed_steps += 1;
+        }
+    }
+
+    const Ctrl& c = *h->mailbox;
+    if (c.error != 0)
+        return MPT_ERR_DEVICE_CHECK;
+
+    mpt_step_result r{};
+    r.found_inf = c.found_inf;
+    r.clipped = c.clipped;
+    r.grad_norm = c.norm;
+    r.clip_coef = c.coef;
+    r.n_zero = c.zero_acc;
+    r.n_subnormal = c.subnormal_acc;
+    r.n_nonfinite = c.n_nonfinite;
+    r.n_fp16_stale = stale ? c.stale_acc : 0;
+    int32_t clean = h->clean_run;
+    r.new_scale = next_scale(h->cfg, c.found_inf != 0, scale, clean);
+    r.clean_run = clean;
+
+    h->scale = r.new_scale;
+    h->clean_run = clean;
+    h->stats.steps += 1;
+    h->stats.skipped += c.found_inf ? 1 : 0;
+    h->stats.scale = h->scale;
+    h->stats.clean_run = clean;
+    h->stats.last = r;
+    h->stats.n_fp16_stale_total += r.n_fp16_stale;
+    *out = r;
+    return MPT_OK;
+}
+
+int mpt_stats(const mpt_handle* h, mpt_stats_t* out)
+{
+    if (!h || !out)
+        return MPT_ERR_INVALID_ARG;
+    *out = h->stats;
+    return MPT_OK;
+}
+
+int mpt_get_scaler_state(const mpt_handle* h, float* scale, int32_t* clean_run)
+{
+    if (!h || !scale || !clean_run)
+        return MPT_ERR_INVALID_ARG;
+    *scale = h->scale;
+    *clean_run = h->clean_run;
+    return MPT_OK;
+}
+
+int mpt_set_scaler_state(mpt_handle* h, float scale, int32_t clean_run)
+{
+    if (!h || !finite(scale) || !(scale > 0.0f) || clean_run < 0)
+        return MPT_ERR_INVALID_ARG;
+    h->scale = scale;
+    h->clean_run = clean_run;
+    h->stats.scale = scale;
+    h->stats.clean_run = clean_run;
+    return MPT_OK;
+}
+
+int mpt_set_timing(mpt_handle* h, int32_t enable)
+{
+    if (!h)
+        return MPT_ERR_INVALID_ARG;
+    if (enable && !h->ev[0]) {
+        for (cudaEvent_t& e : h->ev) {
+            if (cudaEventCreate(&e) != cudaSuccess) {
+                cudaGetLastError();
+                return MPT_ERR_CUDA;
+            }
+        }
+    }
+    h->timing = enable != 0;
+    return MPT_OK;
+}
+
+int mpt_destroy(mpt_handle* h)
+{
+    release(h);
+    return MPT_OK;
+}
+
+const char* mpt_error_string(int code)
+{
+    switch (code) {
+    case MPT_OK: return "ok";
+    case MPT_ERR_INVALID_ARG: return "invalid argument";
+    case MPT_ERR_WORKSPACE: return "workspace too small, misaligned or not device memory";
+    case MPT_ERR_CUDA: return "CUDA runtime error";
+    case MPT_ERR_DEVICE_CHECK: return "checked mode found an out-of-bounds work-table entry";
+    case MPT_ERR_BROKEN: return "handle unusable after an earlier CUDA error";
+    default: return "unknown status";
+    }
+}
+
+}  // extern "C"

@@ -1,0 +1,74 @@
+// mpt_internal.h -- work tables and the device control block of libmpt,
+// shared by the host side (mpt.cu) and the kernels (mpt_kernels.cuh).
+#pragma once
+
+#include <stdint.h>
+
+namespace mpt {
+
+constexpr int kThreads = 256;              // threads per CTA of every kernel
+constexpr int kWarps = kThreads / 32;
+constexpr int kArenaAlign = 16;            // elements: 64 B FP32, 32 B FP16
+constexpr int kDefaultChunk = 32768;       // elements per work bin
+constexpr int kChunkQuantum = 2048;        // chunk sizes are multiples of this
+constexpr int kMaxChunk = 1 << 20;
+constexpr int kSmallTensor = 1024;         // tensors up to this size are packed
+constexpr int kMaxPackedSegs = 1024;       // tensors per packed bin
+
+enum BinKind : int32_t {
+    kChunkBin = 0,   // one contiguous range of one tensor (vectorised)
+    kPackedBin = 1,  // several whole small tensors (flattened, scalar)
+};
+
+// One contiguous range of one tensor.
+struct __align__(16) Seg {
+    int64_t tensor_begin;  // first element, counted inside the tensor
+    int64_t arena_begin;   // the same element's index in the three arenas
+    int32_t tensor;        // index into the gradient-pointer table
+    int32_t len;           // elements
+    int32_t local_begin;   // offset of this range inside its bin
+    int32_t pad;
+};
+
+// The work of one CTA.
+struct __align__(16) Bin {
+    int32_t first_seg;
+    int32_t n_segs;
+    int32_t n_elems;
+    int32_t kind;
+};
+
+// Per-tensor bounds, read by checked mode only.
+struct __align__(16) TensorInfo {
+    int64_t size;
+    int64_t arena_off;
+};
+
+// Device control block.  The check kernel accumulates into the *_acc fields,
+// and its last CTA turns them into the step result, then clears every
+// accumulator (its own and the update kernel's) for the next step.
+struct __align__(16) Ctrl {
+    // check-kernel accumulators
+    unsigned long long nonfinite_acc;
+    unsigned int ticket;
+    unsigned int error_acc;
+    // update-kernel accumulators (cleared by the check kernel's last CTA)
+    unsigned long long zero_acc;
+    unsigned long long subnormal_acc;
+    unsigned long long stale_acc;
+    // step result written by the check kernel's last CTA
+    double sumsq;
+    double norm;
+    unsigned long long n_nonfinite;
+    int32_t found_inf;
+    int32_t clipped;
+    float coef;
+    unsigned int error;    // checked-mode error bits of both kernels
+};
+
+enum ErrorBits : unsigned int {
+    kErrBadBin = 1u,
+    kErrBadSeg = 2u,
+};
+
+}  // namespace mpt

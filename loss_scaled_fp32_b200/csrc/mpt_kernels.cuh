@@ -1,0 +1,600 @@
+// mpt_kernels.cuh -- sm_100a kernels of the loss-scaled FP32-master step.
+//
+//   check_kernel   one pass over the FP16 gradients: overflow check (Step 6 of
+//                  "The Integrated Training Procedure (Figure 1)"), sum of
+//                  squares of the unscaled gradients (global-L2 clip), with a
+//                  deterministic last-CTA finish that writes the step result
+//   update_kernel  the fused per-element update (Steps 5 and 7, weight decay,
+//                  clip, FP16 copy); on an overflow step it only counts
+//   refresh_kernel FP16 copy = round-to-nearest-even(master) (Step 1)
+//
+// All three are HBM-bound streaming kernels on the CUDA cores: there is no
+// contraction, so no tensor-core path.  Per parameter the check reads 2 B and
+// the update reads 10 B and writes 10 B.
+#pragma once
+
+#include <cuda_fp16.h>
+#include <stdint.h>
+
+#include "mpt_internal.h"
+
+namespace mpt {
+
+// ---------------------------------------------------------------------------
+// arguments
+// ---------------------------------------------------------------------------
+
+struct Tables {
+    const Bin* bins;
+    const Seg* segs;
+    const TensorInfo* tensors;
+    const uint16_t* const* grads;  // device table: one FP16 gradient pointer per tensor
+    int32_t nbins;
+    int32_t nsegs;
+    int32_t ntensors;
+    int32_t pad;
+    int64_t arena_total;
+};
+
+struct CheckArgs {
+    Tables t;
+    double* partials;  // one binary64 partial sum of squares per bin
+    Ctrl* ctrl;
+    float inv_scale;   // binary32 1/S
+    float clip;        // <= 0: off
+    double dscale;     // power-of-two S only: 2^1008 / S (see sq_bits)
+};
+
+struct UpdateArgs {
+    Tables t;
+    float* master;
+    float* momentum;
+    uint16_t* w16;
+    Ctrl* ctrl;
+    float inv_scale;
+    float lr;
+    float mu;
+    float wd;
+};
+
+// ---------------------------------------------------------------------------
+// small helpers
+// ---------------------------------------------------------------------------
+
+__device__ __forceinline__ bool seg_ok(const Seg& s, const Tables& t)
+{
+    if (s.tensor < 0 || s.tensor >= t.ntensors || s.len < 0 || s.tensor_begin < 0)
+        return false;
+    const TensorInfo ti = t.tensors[s.tensor];
+    return s.tensor_begin + s.len <= ti.size && s.arena_begin == ti.arena_off + s.tensor_begin &&
+           s.arena_begin + s.len <= t.arena_total;
+}
+
+// Checked mode: validate a bin and all of its ranges before touching memory.
+__device__ __forceinline__ bool bin_ok(const Bin& bin, const Tables& t)
+{
+    if (bin.first_seg < 0 || bin.n_segs < 1 || bin.n_segs > kMaxPackedSegs ||
+        bin.first_seg + bin.n_segs > t.nsegs || bin.n_elems < 0)
+        return false;
+    if (bin.kind == kChunkBin) {
+        const Seg s = t.segs[bin.first_seg];
+        return bin.n_segs == 1 && s.len == bin.n_elems && s.local_begin == 0 && seg_ok(s, t);
+    }
+    if (bin.kind != kPackedBin)
+        return false;
+    int32_t expect = 0;
+    for (int k = 0; k < bin.n_segs; ++k) {
+        const Seg s = t.segs[bin.first_seg + k];
+        if (s.local_begin != expect || !seg_ok(s, t))
+            return false;
+        expect += s.len;
+    }
+    return expect == bin.n_elems;
+}
+
+// Index of the range of a packed bin that holds flattened element j: the
+// last k with begin[k] <= j (begin[] ascending, begin[0] == 0).
+__device__ __forceinline__ int find_seg(const int32_t* begin, int n, int j)
+{
+    int lo = 0, hi = n - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (begin[mid] <= j)
+            lo = mid;
+        else
+            hi = mid - 1;
+    }
+    return lo;
+}
+
+__device__ __forceinline__ uint32_t h2_bits(__half2 h)
+{
+    return *reinterpret_cast<uint32_t*>(&h);
+}
+
+// ---------------------------------------------------------------------------
+// check kernel: overflow flag + sum of squares of the unscaled gradients
+// ---------------------------------------------------------------------------
+
+struct SqAcc {
+    double a0 = 0.0, a1 = 0.0;
+    uint32_t nf = 0;  // bit 15 or 31 set <=> some element seen was +-inf/NaN
+};
+
+// Square of one unscaled gradient, accumulated in binary64.
+//
+// Power-of-two S: x = fp32(g16) * (1/S) is exact, so x can be formed in
+// binary64 straight from the binary16 bits.  The 15 magnitude bits are placed
+// in the high word of a binary64 so that its exponent field is the binary16
+// exponent field and its top fraction bits are the binary16 fraction; that
+// number is the binary16 value times 2^-1008 (binary16 subnormals become
+// binary64 subnormals with the same scale), and one multiply by 2^1008 / S
+// gives x exactly.  The square of an 11-bit significand is exact, so the FMA
+// rounds once, like the sum x*x + acc of the definition.
+//
+// Other S: x is rounded to binary32 first, as the definition says.
+template <bool kPow2>
+__device__ __forceinline__ void sq_bits(uint32_t mag_hi_word, uint16_t h, const CheckArgs& a,
+                                        double& acc)
+{
+    if constexpr (kPow2) {
+        const double x = __hiloint2double((int)mag_hi_word, 0) * a.dscale;
+        acc = fma(x, x, acc);
+    } else {
+        const double x = (double)__fmul_rn(__half2float(__ushort_as_half(h)), a.inv_scale);
+        acc = fma(x, x, acc);
+    }
+}
+
+template <bool kPow2>
+__device__ __forceinline__ void sq_word(uint32_t w, const CheckArgs& a, SqAcc& s)
+{
+    sq_bits<kPow2>((w << 10) & 0x01FFFC00u, (uint16_t)(w & 0xFFFFu), a, s.a0);
+    sq_bits<kPow2>((w >> 6) & 0x01FFFC00u, (uint16_t)(w >> 16), a, s.a1);
+    // Lane is +-inf/NaN <=> its exponent bits are all ones <=> (~w & 0x7C00)
+    // is 0 in that lane; subtracting 0x0400 per lane then borrows into bit 15
+    // (bit 31).  A borrow out of the low lane only reaches the high lane when
+    // the low lane is itself non-finite, so the flag is exact.
+    s.nf |= (~w & 0x7C007C00u) - 0x04000400u;
+}
+
+template <bool kPow2>
+__device__ __forceinline__ void sq_half(uint16_t h, const CheckArgs& a, SqAcc& s)
+{
+    sq_bits<kPow2>(((uint32_t)h << 10) & 0x01FFFC00u, h, a, s.a0);
+    s.nf |= (~(uint32_t)h & 0x7C00u) - 0x0400u;
+}
+
+template <bool kPow2>
+__device__ __forceinline__ void sq_vec(uint4 v, const CheckArgs& a, SqAcc& s)
+{
+    sq_word<kPow2>(v.x, a, s);
+    sq_word<kPow2>(v.y, a, s);
+    sq_word<kPow2>(v.z, a, s);
+    sq_word<kPow2>(v.w, a, s);
+}
+
+template <bool kPow2>
+__device__ __forceinline__ void sq_vec(uint2 v, const CheckArgs& a, SqAcc& s)
+{
+    sq_word<kPow2>(v.x, a, s);
+    sq_word<kPow2>(v.y, a, s);
+}
+
+// One contiguous range: 16-B loads when aligned, 8-B when 8-B aligned, else
+// 2-B loads; unrolled so that every thread has 64 B of loads in flight.
+template <bool kPow2, typename Vec>
+__device__ __forceinline__ void check_range_vec(const uint16_t* g, int len, const CheckArgs& a,
+                                                SqAcc& s)
+{
+    constexpr int kPer = sizeof(Vec) / 2;
+    constexpr int kUnroll = 64 / sizeof(Vec);
+    const Vec* gv = reinterpret_cast<const Vec*>(g);
+    const int nv = len / kPer;
+    int i = threadIdx.x;
+    for (; i + (kUnroll - 1) * kThreads < nv; i += kUnroll * kThreads) {
+        Vec v[kUnroll];
+#pragma unroll
+        for (int k = 0; k < kUnroll; ++k)
+            v[k] = __ldg(gv + i + k * kThreads);
+#pragma unroll
+        for (int k = 0; k < kUnroll; ++k)
+            sq_vec<kPow2>(v[k], a, s);
+    }
+    for (; i < nv; i += kThreads)
+        sq_vec<kPow2>(__ldg(gv + i), a, s);
+    for (int j = nv * kPer + threadIdx.x; j < len; j += kThreads)
+        sq_half<kPow2>(__ldg(g + j), a, s);
+}
+
+template <bool kPow2>
+__device__ __forceinline__ void check_range(const uint16_t* g, int len, const CheckArgs& a,
+                                            SqAcc& s)
+{
+    const uintptr_t p = reinterpret_cast<uintptr_t>(g);
+    if ((p & 15) == 0) {
+        check_range_vec<kPow2, uint4>(g, len, a, s);
+    } else if ((p & 7) == 0) {
+        check_range_vec<kPow2, uint2>(g, len, a, s);
+    } else {
+        int j = threadIdx.x;
+        for (; j + 3 * kThreads < len; j += 4 * kThreads) {
+            uint16_t h[4];
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+                h[k] = __ldg(g + j + k * kThreads);
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+                sq_half<kPow2>(h[k], a, s);
+        }
+        for (; j < len; j += kThreads)
+            sq_half<kPow2>(__ldg(g + j), a, s);
+    }
+}
+
+// Fixed-shape block sum (result valid in thread 0): deterministic for a fixed
+// launch shape, independent of timing.
+__device__ __forceinline__ double block_sum(double x, double* red)
+{
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1)
+        x += __shfl_down_sync(0xffffffffu, x, o);
+    if ((threadIdx.x & 31) == 0)
+        red[threadIdx.x >> 5] = x;
+    __syncthreads();
+    double t = 0.0;
+    if (threadIdx.x == 0) {
+#pragma unroll
+        for (int w = 0; w < kWarps; ++w)
+            t += red[w];
+    }
+    __syncthreads();
+    return t;
+}
+
+__device__ __forceinline__ unsigned int block_sum_u32(unsigned int x, unsigned int* red)
+{
+    x = __reduce_add_sync(0xffffffffu, x);
+    if ((threadIdx.x & 31) == 0)
+        red[threadIdx.x >> 5] = x;
+    __syncthreads();
+    unsigned int t = 0;
+    if (threadIdx.x == 0) {
+#pragma unroll
+        for (int w = 0; w < kWarps; ++w)
+            t += red[w];
+    }
+    __syncthreads();
+    return t;
+}
+
+// Exact count of non-finite elements of a bin (run only by a CTA that saw one).
+__device__ unsigned int count_nonfinite(const Bin& bin, const Tables& t)
+{
+    unsigned int c = 0;
+    for (int k = 0; k < bin.n_segs; ++k) {
+        const Seg s = t.segs[bin.first_seg + k];
+        const uint16_t* g = t.grads[s.tensor] + s.tensor_begin;
+        for (int j = threadIdx.x; j < s.len; j += kThreads)
+            c += ((g[j] & 0x7C00u) == 0x7C00u) ? 1u : 0u;
+    }
+    return c;
+}
+
+template <bool kPow2, bool kChecked>
+__global__ void __launch_bounds__(kThreads) check_kernel(CheckArgs a)
+{
+    __shared__ int32_t s_begin[kMaxPackedSegs];
+    __shared__ double s_red[kWarps];
+    __shared__ unsigned int s_ured[kWarps];
+    __shared__ int s_last;
+
+    const Tables& t = a.t;
+    const Bin bin = t.bins[blockIdx.x];
+    SqAcc s;
+    bool valid = true;
+    if constexpr (kChecked)
+        valid = bin_ok(bin, t);
+
+    if (valid) {
+        if (bin.kind == kChunkBin) {
+            const Seg sg = t.segs[bin.first_seg];
+            check_range<kPow2>(t.grads[sg.tensor] + sg.tensor_begin, sg.len, a, s);
+        } else {
+            for (int k = threadIdx.x; k < bin.n_segs; k += kThreads)
+                s_begin[k] = t.segs[bin.first_seg + k].local_begin;
+            __syncthreads();
+            for (int j = threadIdx.x; j < bin.n_elems; j += kThreads) {
+                const Seg sg = t.segs[bin.first_seg + find_seg(s_begin, bin.n_segs, j)];
+                sq_half<kPow2>(__ldg(t.grads[sg.tensor] + sg.tensor_begin + (j - sg.local_begin)), a, s);
+            }
+        }
+    }
+
+    // Non-finite count: exact, but only computed by a CTA that saw one.
+    unsigned int nf = 0;
+    if (__syncthreads_or((s.nf & 0x80008000u) != 0))
+        nf = block_sum_u32(count_nonfinite(bin, t), s_ured);
+
+    const double part = block_sum(s.a0 + s.a1, s_red);
+    if (threadIdx.x == 0) {
+        a.partials[blockIdx.x] = part;
+        if (nf)
+            atomicAdd(&a.ctrl->nonfinite_acc, (unsigned long long)nf);
+        if (!valid)
+            atomicOr(&a.ctrl->error_acc, (unsigned int)kErrBadBin);
+        __threadfence();
+        const unsigned int ticket = atomicAdd(&a.ctrl->ticket, 1u);
+        s_last = (ticket == gridDim.x - 1);
+    }
+    __syncthreads();
+    if (!s_last)
+        return;
+
+    // Last CTA: every other CTA's partial and counters are visible.  Sum the
+    // partials in bin order with a fixed pattern, then write the result.
+    __threadfence();
+    double x = 0.0;
+    for (int k = threadIdx.x; k < t.nbins; k += kThreads)
+        x += __ldcg(a.partials + k);
+    const double sumsq = block_sum(x, s_red);
+    if (threadIdx.x == 0) {
+        Ctrl* c = a.ctrl;
+        const unsigned long long n_nonfinite = atomicAdd(&c->nonfinite_acc, 0ull);
+        const unsigned int err = atomicOr(&c->error_acc, 0u);
+        const bool found = n_nonfinite != 0;
+        const double norm = found ? __longlong_as_double(0x7ff0000000000000ll) : sqrt(sumsq);
+        const bool clipped = !found && a.clip > 0.0f && norm > (double)a.clip;
+        c->sumsq = sumsq;
+        c->norm = norm;
+        c->n_nonfinite = n_nonfinite;
+        c->found_inf = found ? 1 : 0;
+        c->clipped = clipped ? 1 : 0;
+        c->coef = clipped ? __double2float_rn((double)a.clip / norm) : 1.0f;
+        c->error = err;
+        c->nonfinite_acc = 0;
+        c->error_acc = 0;
+        c->zero_acc = 0;
+        c->subnormal_acc = 0;
+        c->stale_acc = 0;
+        c->ticket = 0;
+    }
+}
+
+// ---------------------------------------------------------------------------
+// update kernel: fused unscale, clip, weight decay, momentum, master, FP16
+// ---------------------------------------------------------------------------
+
+struct UpdParams {
+    float inv_scale, coef, lr, mu, wd;
+};
+
+// One element, each operation rounded to binary32 on its own (no FMA).
+__device__ __forceinline__ void upd1(float g16f, float& w, float& v, const UpdParams& p)
+{
+    float g = __fmul_rn(g16f, p.inv_scale);  // unscale
+    g = __fmul_rn(g, p.coef);                // global-L2 clip (coef 1: exact no-op)
+    const float t = __fmul_rn(p.wd, w);      // weight decay on the FP32 master
+    const float d = __fadd_rn(g, t);
+    const float u = __fmul_rn(p.mu, v);      // momentum
+    v = __fadd_rn(u, d);
+    const float s = __fmul_rn(p.lr, v);      // master update
+    w = __fsub_rn(w, s);
+}
+
+// Lane-packed counters: each 32-bit word carries two 16-bit counts (one per
+// FP16 lane); a thread adds at most 2^12 per lane, far below overflow.
+__device__ __forceinline__ void count_word(uint32_t w, uint32_t& nz2, uint32_t& ns2)
+{
+    const uint32_t m = w & 0x7FFF7FFFu;
+    nz2 += ((m + 0x7FFF7FFFu) >> 15) & 0x00010001u;  // lane != +-0
+    ns2 += ((m + 0x7C007C00u) >> 15) & 0x00010001u;  // lane >= 2^-14 (or inf/NaN)
+}
+
+__device__ __forceinline__ void count_half(uint16_t h, uint32_t& nz2, uint32_t& ns2)
+{
+    const uint32_t m = h & 0x7FFFu;
+    nz2 += m != 0 ? 1u : 0u;
+    ns2 += m >= 0x0400u ? 1u : 0u;
+}
+
+template <bool kStale>
+__device__ __forceinline__ void stale1(float w_old, float w_new, uint32_t& stale)
+{
+    if constexpr (kStale) {
+        if (w_new != w_old &&
+            __half_as_ushort(__float2half_rn(w_new)) == __half_as_ushort(__float2half_rn(w_old)))
+            ++stale;
+    }
+}
+
+// Four elements: 8-B FP16 gradient load, 16-B master and momentum loads,
+// 16-B + 16-B + 8-B stores (every warp access is 256 B or 512 B contiguous).
+template <bool kStale>
+__device__ __forceinline__ void upd4(uint2 g, float4& w, float4& v, uint2& h, const UpdParams& p,
+                                     uint32_t& stale)
+{
+    const float2 g01 = __half22float2(*reinterpret_cast<const __half2*>(&g.x));
+    const float2 g23 = __half22float2(*reinterpret_cast<const __half2*>(&g.y));
+    const float4 w0 = w;
+    upd1(g01.x, w.x, v.x, p);
+    upd1(g01.y, w.y, v.y, p);
+    upd1(g23.x, w.z, v.z, p);
+    upd1(g23.y, w.w, v.w, p);
+    h.x = h2_bits(__floats2half2_rn(w.x, w.y));
+    h.y = h2_bits(__floats2half2_rn(w.z, w.w));
+    stale1<kStale>(w0.x, w.x, stale);
+    stale1<kStale>(w0.y, w.y, stale);
+    stale1<kStale>(w0.z, w.z, stale);
+    stale1<kStale>(w0.w, w.w, stale);
+}
+
+template <bool kStale>
+__device__ __forceinline__ void upd_scalar(uint16_t g16, float* w, float* v, uint16_t* h,
+                                           const UpdParams& p, uint32_t& stale)
+{
+    float wi = *w, vi = *v;
+    const float w0 = wi;
+    upd1(__half2float(__ushort_as_half(g16)), wi, vi, p);
+    __stcs(w, wi);
+    __stcs(v, vi);
+    *h = __half_as_ushort(__float2half_rn(wi));
+    stale1<kStale>(w0, wi, stale);
+}
+
+template <bool kStale>
+__device__ __forceinline__ void update_range(const uint16_t* g, float* w, float* v, uint16_t* h,
+                                             int len, const UpdParams& p, uint32_t& nz2,
+                                             uint32_t& ns2, uint32_t& stale)
+{
+    int start = 0;
+    if ((reinterpret_cast<uintptr_t>(g) & 7) == 0) {
+        constexpr int kUnroll = 4;
+        const uint2* g4 = reinterpret_cast<const uint2*>(g);
+        float4* w4 = reinterpret_cast<float4*>(w);
+        float4* v4 = reinterpret_cast<float4*>(v);
+        uint2* h4 = reinterpret_cast<uint2*>(h);
+        const int nq = len >> 2;
+        int i = threadIdx.x;
+        for (; i + (kUnroll - 1) * kThreads < nq; i += kUnroll * kThreads) {
+            uint2 gq[kUnroll], hq[kUnroll];
+            float4 wq[kUnroll], vq[kUnroll];
+#pragma unroll
+            for (int k = 0; k < kUnroll; ++k) {
+                gq[k] = __ldcs(g4 + i + k * kThreads);
+                wq[k] = __ldcs(w4 + i + k * kThreads);
+                vq[k] = __ldcs(v4 + i + k * kThreads);
+            }
+#pragma unroll
+            for (int k = 0; k < kUnroll; ++k) {
+                upd4<kStale>(gq[k], wq[k], vq[k], hq[k], p, stale);
+                count_word(gq[k].x, nz2, ns2);
+                count_word(gq[k].y, nz2, ns2);
+            }
+#pragma unroll
+            for (int k = 0; k < kUnroll; ++k) {
+                __stcs(w4 + i + k * kThreads, wq[k]);
+                __stcs(v4 + i + k * kThreads, vq[k]);
+                __stcs(h4 + i + k * kThreads, hq[k]);
+            }
+        }
+        for (; i < nq; i += kThreads) {
+            uint2 gq = __ldcs(g4 + i), hq;
+            float4 wq = __ldcs(w4 + i), vq = __ldcs(v4 + i);
+            upd4<kStale>(gq, wq, vq, hq, p, stale);
+            count_word(gq.x, nz2, ns2);
+            count_word(gq.y, nz2, ns2);
+            __stcs(w4 + i, wq);
+            __stcs(v4 + i, vq);
+            __stcs(h4 + i, hq);
+        }
+        start = nq << 2;
+    }
+    for (int j = start + threadIdx.x; j < len; j += kThreads) {
+        const uint16_t gh = __ldcs(g + j);
+        upd_scalar<kStale>(gh, w + j, v + j, h + j, p, stale);
+        count_half(gh, nz2, ns2);
+    }
+}
+
+// Overflow step: the update is skipped; only the range counts are taken.
+__device__ __forceinline__ void count_range(const uint16_t* g, int len, uint32_t& nz2, uint32_t& ns2)
+{
+    int start = 0;
+    if ((reinterpret_cast<uintptr_t>(g) & 15) == 0) {
+        const uint4* gv = reinterpret_cast<const uint4*>(g);
+        const int nv = len >> 3;
+        for (int i = threadIdx.x; i < nv; i += kThreads) {
+            const uint4 q = __ldcs(gv + i);
+            count_word(q.x, nz2, ns2);
+            count_word(q.y, nz2, ns2);
+            count_word(q.z, nz2, ns2);
+            count_word(q.w, nz2, ns2);
+        }
+        start = nv << 3;
+    }
+    for (int j = start + threadIdx.x; j < len; j += kThreads)
+        count_half(__ldcs(g + j), nz2, ns2);
+}
+
+template <bool kStale, bool kChecked>
+__global__ void __launch_bounds__(kThreads) update_kernel(UpdateArgs a)
+{
+    __shared__ int32_t s_begin[kMaxPackedSegs];
+    __shared__ unsigned int s_ured[kWarps];
+
+    const Tables& t = a.t;
+    // Bins run in reverse order: the check kernel read the last bins last, so
+    // their gradients are the ones still resident in L2.
+    const int b = t.nbins - 1 - (int)blockIdx.x;
+    const Bin bin = t.bins[b];
+    bool valid = true;
+    if constexpr (kChecked)
+        valid = bin_ok(bin, t);
+
+    const Ctrl* c = a.ctrl;
+    const bool skip = c->found_inf != 0;
+    const UpdParams p{a.inv_scale, c->coef, a.lr, a.mu, a.wd};
+    uint32_t nz2 = 0, ns2 = 0, stale = 0;
+
+    if (valid) {
+        if (bin.kind == kChunkBin) {
+            const Seg sg = t.segs[bin.first_seg];
+            const uint16_t* g = t.grads[sg.tensor] + sg.tensor_begin;
+            if (skip)
+                count_range(g, sg.len, nz2, ns2);
+            else
+                update_range<kStale>(g, a.master + sg.arena_begin, a.momentum + sg.arena_begin,
+                                     a.w16 + sg.arena_begin, sg.len, p, nz2, ns2, stale);
+        } else {
+            for (int k = threadIdx.x; k < bin.n_segs; k += kThreads)
+                s_begin[k] = t.segs[bin.first_seg + k].local_begin;
+            __syncthreads();
+            for (int j = threadIdx.x; j < bin.n_elems; j += kThreads) {
+                const Seg sg = t.segs[bin.first_seg + find_seg(s_begin, bin.n_segs, j)];
+                const int64_t off = j - sg.local_begin;
+                const uint16_t gh = __ldcs(t.grads[sg.tensor] + sg.tensor_begin + off);
+                count_half(gh, nz2, ns2);
+                if (!skip) {
+                    const int64_t e = sg.arena_begin + off;
+                    upd_scalar<kStale>(gh, a.master + e, a.momentum + e, a.w16 + e, p, stale);
+                }
+            }
+        }
+    }
+
+    const unsigned int nz = block_sum_u32((nz2 & 0xFFFFu) + (nz2 >> 16), s_ured);
+    const unsigned int ns = block_sum_u32((ns2 & 0xFFFFu) + (ns2 >> 16), s_ured);
+    unsigned int st = 0;
+    if constexpr (kStale)
+        st = block_sum_u32(stale, s_ured);
+    if (threadIdx.x == 0) {
+        Ctrl* cw = a.ctrl;
+        if (valid) {
+            atomicAdd(&cw->zero_acc, (unsigned long long)(bin.n_elems - nz));
+            atomicAdd(&cw->subnormal_acc, (unsigned long long)(nz - ns));
+            if (st)
+                atomicAdd(&cw->stale_acc, (unsigned long long)st);
+        } else {
+            atomicOr(&cw->error, (unsigned int)kErrBadBin);
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
+// refresh kernel: FP16 working copy from the FP32 master
+// ---------------------------------------------------------------------------
+
+__global__ void __launch_bounds__(kThreads) refresh_kernel(const float4* master, uint2* w16, int64_t n4)
+{
+    const int64_t stride = (int64_t)gridDim.x * kThreads;
+    for (int64_t i = (int64_t)blockIdx.x * kThreads + threadIdx.x; i < n4; i += stride) {
+        const float4 m = __ldcs(master + i);
+        uint2 o;
+        o.x = h2_bits(__floats2half2_rn(m.x, m.y));
+        o.y = h2_bits(__floats2half2_rn(m.z, m.w));
+        __stcs(w16 + i, o);
+    }
+}
+
+}  // namespace mpt

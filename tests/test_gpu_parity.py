@@ -1,0 +1,212 @@
+"""GPU parity: libmpt (through its C ABI) against the CPU oracle, element by
+element, on seeded inputs shaped like the five workloads, at sizes the oracle
+finishes in seconds (several work bins and ragged tails each)."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads as W
+from workloads.configs import Config as WConfig, TensorSpec, miniature
+from loss_scaled_fp32_b200 import MPT, Config, MPT_FLAG_CHECKED, MPT_FLAG_COUNT_STALE
+
+from parity import Pair
+
+pytestmark = pytest.mark.gpu
+
+
+def custom(sizes, law=("log2_uniform", -30.0, -6.0), scale0=1024.0, growth_interval=0,
+           clip=0.0, steps=3, seed=7, lr=0.01, momentum=0.9, weight_decay=1e-4, injections=None):
+    tensors = [TensorSpec(f"t{i}", (int(s),), ("normal", 0.05)) for i, s in enumerate(sizes)]
+    return WConfig(name="custom", tensors=tensors, grad_law=law, scale0=scale0,
+                   growth_interval=growth_interval, lr=lr, momentum=momentum,
+                   weight_decay=weight_decay, clip=clip, steps=steps, seed=seed,
+                   injections=injections or (lambda step: []))
+
+
+# ---------------------------------------------------------------------------
+# the five workloads (reduced where the oracle would take minutes)
+# ---------------------------------------------------------------------------
+
+def test_flat1m_full_with_overflow_step():
+    cfg = W.get("flat1m")
+    p = Pair(cfg)
+    scales = []
+    for _ in range(cfg.steps):
+        r, _ = p.step()
+        scales.append(r["new_scale"])
+    assert scales == [1024.0] * 4 + [512.0] * 6          # backoff at step 5, no growth
+    assert p.bitexact_steps == cfg.steps + 1
+
+
+def test_resnet50_first_steps():
+    cfg = W.get("resnet50")
+    p = Pair(cfg)
+    for _ in range(3):
+        r, _ = p.step()
+        assert r["found_inf"] == 0
+    assert p.bitexact_steps == 4
+
+
+def test_gpt2_medium_sample_dynamic_scale_and_clip():
+    cfg = miniature("gpt2_medium")
+    p = Pair(cfg)
+    clipped = 0
+    for i in range(8):
+        # a threshold below the norm of the sample exercises the clip path
+        r, ro = p.step(clip=0.05)
+        clipped += r["clipped"]
+    assert clipped > 0
+
+
+def test_gpt_1p3b_sample():
+    cfg = miniature("gpt_1p3b")
+    p = Pair(cfg)
+    for _ in range(3):
+        p.step()
+
+
+def test_ragged_sample_with_unaligned_pointers_and_injections():
+    full = W.get("ragged20k")
+    sizes = W.configs.ragged_sizes(n=3000, seed=11, log_max=14)
+    plan = {2: [(5, 0, 0x7C00)], 4: [(100, int(sizes[100]) - 1, 0xFC00)],
+            7: [(2999, int(sizes[2999]) // 2, 0x7E00)]}
+    cfg = custom(sizes, law=full.grad_law, scale0=2.0 ** 10, growth_interval=4, steps=10,
+                 injections=lambda s: plan.get(s, []))
+    shifted = set(range(0, 3000, 3))
+    p = Pair(cfg, shifted=shifted)
+    found = []
+    for _ in range(cfg.steps):
+        r, _ = p.step()
+        found.append(r["found_inf"])
+    assert found[1] == 1 and found[3] == 1 and found[6] == 1
+
+
+# ---------------------------------------------------------------------------
+# edge cases
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("sizes", [[1], [2, 3], list(range(1, 18)), [7] * 5000,
+                                   [1024, 1025, 1023], [32768], [32769, 32767, 65536 + 5],
+                                   [200_003]])
+def test_edge_sizes(sizes):
+    p = Pair(custom(sizes, steps=2))
+    p.step()
+    p.step()
+
+
+@pytest.mark.parametrize("shift", [0, 1, 2, 3, 4, 5, 6, 7])
+def test_unaligned_gradient_pointers(shift):
+    # 2-, 4-, 6-, 8-, ... byte offsets select the 16-B, 8-B and 2-B load paths
+    cfg = custom([10_000, 70_001, 33], steps=2)
+    p = Pair(cfg)
+    for step in (1, 2):
+        host = p.grads(step, p.scale)
+        # every tensor placed `shift` elements after its aligned offset
+        flat = torch.zeros(p.layout.total + 64, dtype=torch.int16, device="cuda")
+        views = []
+        for off, n, hv in zip(p.layout.offsets, p.layout.sizes, p.layout.views(host)):
+            flat[off + shift: off + shift + n].copy_(hv)
+            views.append(flat[off + shift: off + shift + n])
+        p.step(host=host, gpu_grads=views)
+
+
+@pytest.mark.parametrize("scale", [1000.0, 3.0, 2.0 ** -20, 2.0 ** 40, 0.7])
+def test_non_power_of_two_and_extreme_scales(scale):
+    cfg = custom([50_000, 999, 4097], law=("log2_uniform", -40.0, -20.0), scale0=scale, steps=2)
+    p = Pair(cfg)
+    p.step()
+    p.step()
+
+
+def test_checked_mode_and_stale_counts():
+    cfg = custom([100_000, 17, 3000], steps=3, lr=1e-3)
+    p = Pair(cfg, flags=MPT_FLAG_CHECKED | MPT_FLAG_COUNT_STALE)
+    for _ in range(3):
+        r, ro = p.step()
+        assert r["n_fp16_stale"] == ro["n_stale"]
+        assert r["n_fp16_stale"] > 0
+
+
+@pytest.mark.parametrize("chunk", [2048, 4096, 1 << 20])
+def test_chunk_sizes(chunk):
+    cfg = custom([300_000, 5, 2049, 100_000], steps=2)
+    p = Pair(cfg, chunk=chunk)
+    p.step()
+    p.step()
+
+
+@pytest.mark.parametrize("pattern", [0x7C00, 0xFC00, 0x7E00, 0x7C01, 0xFFFF])
+def test_overflow_leaves_state_bitwise_unchanged(pattern):
+    cfg = custom([40_000, 3, 1500], steps=2)
+    p = Pair(cfg)
+    p.step()
+    before = [x.copy() for x in sum(p.gpu_state(), [])]
+    host = p.grads(2, p.scale)
+    host[p.layout.offsets[2] + 1499] = pattern - 65536 if pattern >= 0x8000 else pattern
+    r, _ = p.step(host=host)
+    assert r["found_inf"] == 1 and r["n_nonfinite"] == 1 and math.isinf(r["grad_norm"])
+    after = sum(p.gpu_state(), [])
+    assert all(a.tobytes() == b.tobytes() for a, b in zip(before, after))
+
+
+def test_all_zero_and_all_subnormal_gradients():
+    cfg = custom([10_000, 333], steps=1)
+    p = Pair(cfg)
+    host = torch.zeros(p.layout.total, dtype=torch.int16)
+    r, _ = p.step(host=host)
+    assert r["n_zero"] == 10_333 and r["grad_norm"] == 0.0
+    host = torch.full((p.layout.total,), 0x0123, dtype=torch.int16)
+    r, _ = p.step(host=host)
+    assert r["n_subnormal"] == 10_333
+
+
+def test_determinism_bitwise():
+    cfg = miniature("gpt2_medium")
+    runs = []
+    for _ in range(2):
+        p = Pair(cfg)
+        out = [p.step(clip=0.05)[0]["grad_norm"] for _ in range(3)]
+        runs.append((out, [x.tobytes() for x in sum(p.gpu_state(), [])]))
+    assert runs[0] == runs[1]
+
+
+def test_checkpoint_resume_matches_straight_run():
+    cfg = custom([123_457, 64, 4096], growth_interval=2, scale0=2.0 ** 14, steps=10,
+                 law=("log2_uniform", -24.0, 1.0))
+    straight = Pair(cfg)
+    for _ in range(10):
+        straight.step()
+    a = Pair(cfg)
+    for _ in range(5):
+        a.step()
+    # save: master + momentum (the workspace arenas) and the scaler state
+    saved = [(a.opt.master(i).clone(), a.opt.momentum(i).clone()) for i in range(3)]
+    scale, clean = a.opt.scaler_state()
+    b = Pair(cfg)
+    for i, (m, v) in enumerate(saved):
+        b.opt.master(i).copy_(m)
+        b.opt.momentum(i).copy_(v)
+    b.opt.refresh_half()
+    b.opt.set_scaler_state(scale, clean)
+    b.state, b.scale, b.step_no = a.state, scale, 5
+    for _ in range(5):
+        b.step()
+    s1 = [x.tobytes() for x in sum(straight.gpu_state(), [])]
+    s2 = [x.tobytes() for x in sum(b.gpu_state(), [])]
+    assert s1 == s2
+    assert straight.opt.scaler_state() == b.opt.scaler_state()
+
+
+def test_stats_and_timing():
+    cfg = custom([70_000], steps=3)
+    p = Pair(cfg)
+    p.opt.set_timing(True)
+    for _ in range(3):
+        p.step()
+    st = p.opt.stats()
+    assert st["steps"] == 3 and st["timed_steps"] == 3
+    assert st["check_ms_total"] > 0 and st["update_ms_total"] > 0
+    assert st["scale"] == p.scale
