@@ -56,6 +56,8 @@ extern "C" {
 #define MPT_ERR_DEVICE_CHECK (-4) /* checked mode found a work-table entry out
                                      of bounds; that entry was not touched   */
 #define MPT_ERR_BROKEN (-5)       /* the handle saw MPT_ERR_CUDA earlier     */
+#define MPT_ERR_TOO_LARGE (-6)    /* input longer than MPT_NOALLOC_MAX_ELEMS
+                                     (mpt_check_flat_noalloc only)           */
 
 /* ---- configuration ------------------------------------------------------ */
 #define MPT_FLAG_CHECKED 0x1u     /* kernels validate every work-table entry
@@ -178,6 +180,54 @@ int mpt_destroy(mpt_handle* h);
 
 /* Static description of a status code (never NULL). */
 const char* mpt_error_string(int code);
+
+/* ---- allocation-free check of one flat gradient buffer ------------------ */
+
+/* The paper has no counterpart to this call: it serves callers of this
+ * library, not a step of the method.
+ *
+ * Some callers cannot allocate device memory: a library loaded into a host
+ * program whose memory pool already owns the device (a cudaMalloc there
+ * fails, or takes memory the host program has counted on), and code whose
+ * step loop must never enter the CUDA allocator (cudaMalloc and cudaFree can
+ * synchronize the device and stall every stream).  mpt_step needs a
+ * workspace allocated up front; this call needs none.  It runs the overflow
+ * check and the global norm of the step (found_inf, the L2 norm of the
+ * unscaled gradients, the clip coefficient, the count of +-inf/NaN) over ONE
+ * contiguous FP16 buffer, keeping its scratch (one binary64 partial per
+ * 32768 elements and two counters, about 256 KiB) in a fixed array inside the
+ * library that every GPU which loads the library holds until the process
+ * exits.
+ *
+ *   d_grads_half  device pointer to n binary16 gradients (2-byte aligned),
+ *                 scaled by `scale`; only read
+ *   n             1 <= n <= MPT_NOALLOC_MAX_ELEMS; longer inputs return
+ *                 MPT_ERR_TOO_LARGE before any CUDA call
+ *   scale, clip   as in mpt_step (clip <= 0: no clipping, coefficient 1)
+ *   d_result      device pointer (8-byte aligned) that receives the
+ *                 mpt_check_result when the queued work completes
+ *   cuda_stream   stream to queue on; the call returns without waiting
+ *
+ * The first call on each device looks up the device address of the scratch
+ * array (with that device current); make that first call before any stream
+ * capture.  Every call on a device shares the one scratch array, which keeps
+ * the last call's contents; each call clears the counters it needs before its
+ * kernel runs.  Calls whose work overlaps on the GPU (other streams, other
+ * host threads) race on that array and give wrong results: serialize them.
+ * Errors: MPT_ERR_INVALID_ARG, MPT_ERR_TOO_LARGE, MPT_ERR_CUDA. */
+#define MPT_NOALLOC_MAX_ELEMS (((int64_t)1) << 30)
+
+typedef struct {
+    int32_t found_inf;     /* 1: some gradient was +-inf/NaN                     */
+    int32_t clipped;       /* 1: clip > 0 and grad_norm > clip                   */
+    double grad_norm;      /* L2 norm of the unscaled gradients; +inf if found   */
+    float clip_coef;       /* clip / grad_norm when clipped, else 1              */
+    int32_t reserved;
+    uint64_t n_nonfinite;  /* gradients that are +-inf or NaN                    */
+} mpt_check_result;
+
+int mpt_check_flat_noalloc(const void* d_grads_half, int64_t n, float scale, float clip,
+                           mpt_check_result* d_result, void* cuda_stream);
 
 #ifdef __cplusplus
 }

@@ -18,7 +18,7 @@ import os
 
 from . import build as _build
 
-__all__ = ["MPT", "Config", "MptError", "lib", "grad_pointers",
+__all__ = ["MPT", "Config", "MptError", "lib", "grad_pointers", "check_flat_noalloc",
            "MPT_FLAG_CHECKED", "MPT_FLAG_COUNT_STALE"]
 
 MPT_FLAG_CHECKED = 0x1
@@ -30,6 +30,8 @@ MPT_ERR_WORKSPACE = -2
 MPT_ERR_CUDA = -3
 MPT_ERR_DEVICE_CHECK = -4
 MPT_ERR_BROKEN = -5
+MPT_ERR_TOO_LARGE = -6
+MPT_NOALLOC_MAX_ELEMS = 1 << 30
 
 
 class MptError(RuntimeError):
@@ -60,6 +62,16 @@ class StepResult(ctypes.Structure):
                 ("reserved", ctypes.c_int32), ("n_zero", ctypes.c_uint64),
                 ("n_subnormal", ctypes.c_uint64), ("n_nonfinite", ctypes.c_uint64),
                 ("n_fp16_stale", ctypes.c_uint64)]
+
+    def as_dict(self):
+        return {k: getattr(self, k) for k, _ in self._fields_ if k != "reserved"}
+
+
+class CheckResult(ctypes.Structure):
+    """``mpt_check_result``: what mpt_check_flat_noalloc writes to device memory."""
+    _fields_ = [("found_inf", ctypes.c_int32), ("clipped", ctypes.c_int32),
+                ("grad_norm", ctypes.c_double), ("clip_coef", ctypes.c_float),
+                ("reserved", ctypes.c_int32), ("n_nonfinite", ctypes.c_uint64)]
 
     def as_dict(self):
         return {k: getattr(self, k) for k, _ in self._fields_ if k != "reserved"}
@@ -102,6 +114,7 @@ def lib():
             "mpt_set_scaler_state": [vp, f32, i32],
             "mpt_set_timing": [vp, i32],
             "mpt_destroy": [vp],
+            "mpt_check_flat_noalloc": [vp, ctypes.c_int64, f32, f32, vp, vp],
         }
         for name, args in sig.items():
             fn = getattr(L, name)
@@ -121,6 +134,20 @@ def _check(code, what):
 def grad_pointers(tensors):
     """Host array of device pointers (build once, reuse across steps)."""
     return (ctypes.c_void_p * len(tensors))(*[t.data_ptr() for t in tensors])
+
+
+def check_flat_noalloc(grads, scale, clip, out, stream=None):
+    """Queue ``mpt_check_flat_noalloc`` on one contiguous FP16 CUDA tensor;
+    ``out`` is a CUDA tensor of at least ``ctypes.sizeof(CheckResult)`` bytes
+    that receives the result.  Returns without waiting."""
+    if not grads.is_contiguous() or grads.element_size() != 2:
+        raise ValueError("grads must be one contiguous 2-byte tensor")
+    if out.numel() * out.element_size() < ctypes.sizeof(CheckResult):
+        raise ValueError("out is too small for mpt_check_result")
+    _check(lib().mpt_check_flat_noalloc(ctypes.c_void_p(grads.data_ptr()), grads.numel(),
+                                        scale, clip, ctypes.c_void_p(out.data_ptr()),
+                                        _stream_ptr(stream, grads.device)),
+           "mpt_check_flat_noalloc")
 
 
 def _stream_ptr(stream, device):

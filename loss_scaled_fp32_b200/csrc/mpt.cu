@@ -14,6 +14,7 @@
 #include <cmath>
 #include <cstdlib>
 #include <cstring>
+#include <mutex>
 #include <new>
 #include <vector>
 
@@ -547,8 +548,159 @@ const char* mpt_error_string(int code)
     case MPT_ERR_CUDA: return "CUDA runtime error";
     case MPT_ERR_DEVICE_CHECK: return "checked mode found an out-of-bounds work-table entry";
     case MPT_ERR_BROKEN: return "handle unusable after an earlier CUDA error";
+    case MPT_ERR_TOO_LARGE: return "input longer than MPT_NOALLOC_MAX_ELEMS (2^30) elements";
     default: return "unknown status";
     }
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Allocation-free check of one flat FP16 buffer (mpt_check_flat_noalloc).
+//
+// The same per-CTA work as check_kernel (check_range, block sums, exact
+// non-finite count, last-CTA fixed-order finish), over bins cut from one
+// contiguous buffer by block index, so no work tables are needed.  Its scratch
+// -- two counters and one binary64 partial per bin -- lives in the file-scope
+// array below instead of a caller workspace.
+// ---------------------------------------------------------------------------
+
+namespace {
+
+constexpr int kNoAllocChunk = kDefaultChunk;
+constexpr int64_t kNoAllocMaxBins = MPT_NOALLOC_MAX_ELEMS / kNoAllocChunk;
+constexpr size_t kNoAllocCtrlBytes = 256;
+constexpr size_t kNoAllocScratchBytes = kNoAllocCtrlBytes + sizeof(double) * kNoAllocMaxBins;
+constexpr int kNoAllocMaxDevices = 64;
+
+struct NoAllocCtrl {
+    unsigned long long nonfinite_acc;
+    unsigned int ticket;
+    unsigned int pad;
+};
+static_assert(sizeof(NoAllocCtrl) <= kNoAllocCtrlBytes, "counters fit their slot");
+static_assert(MPT_NOALLOC_MAX_ELEMS % kNoAllocChunk == 0, "whole bins");
+
+// Host-side lookup of the scratch array's device address, once per device.
+std::once_flag g_noalloc_once[kNoAllocMaxDevices];
+unsigned char* g_noalloc_addr[kNoAllocMaxDevices];
+cudaError_t g_noalloc_status[kNoAllocMaxDevices];
+
+}  // namespace
+
+// About 256 KiB on every device that loads the library, held until exit.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+template <bool kPow2>
+__global__ void __launch_bounds__(kThreads)
+check_flat_kernel(const uint16_t* g, int64_t n, unsigned char* scratch, mpt_check_result* out,
+                  float inv_scale, double dscale, float clip)
+{
+    __shared__ double s_red[kWarps];
+    __shared__ unsigned int s_ured[kWarps];
+    __shared__ int s_last;
+
+    NoAllocCtrl* c = reinterpret_cast<NoAllocCtrl*>(scratch);
+    double* partials = reinterpret_cast<double*>(scratch + kNoAllocCtrlBytes);
+    const int64_t begin = (int64_t)blockIdx.x * kNoAllocChunk;
+    const int len = (int)(n - begin < kNoAllocChunk ? n - begin : kNoAllocChunk);
+
+    CheckArgs a{};
+    a.inv_scale = inv_scale;
+    a.dscale = dscale;
+    a.clip = clip;
+    SqAcc s;
+    check_range<kPow2>(g + begin, len, a, s);
+
+    unsigned int nf = 0;
+    if (__syncthreads_or((s.nf & 0x80008000u) != 0)) {
+        unsigned int cnt = 0;
+        for (int j = threadIdx.x; j < len; j += kThreads)
+            cnt += ((g[begin + j] & 0x7C00u) == 0x7C00u) ? 1u : 0u;
+        nf = block_sum_u32(cnt, s_ured);
+    }
+    const double part = block_sum(s.a0 + s.a1, s_red);
+    if (threadIdx.x == 0) {
+        partials[blockIdx.x] = part;
+        if (nf)
+            atomicAdd(&c->nonfinite_acc, (unsigned long long)nf);
+        __threadfence();
+        s_last = (atomicAdd(&c->ticket, 1u) == gridDim.x - 1);
+    }
+    __syncthreads();
+    if (!s_last)
+        return;
+
+    __threadfence();
+    double x = 0.0;
+    for (int k = threadIdx.x; k < (int)gridDim.x; k += kThreads)
+        x += __ldcg(partials + k);
+    const double sumsq = block_sum(x, s_red);
+    if (threadIdx.x == 0) {
+        const unsigned long long nnf = atomicAdd(&c->nonfinite_acc, 0ull);
+        const bool found = nnf != 0;
+        const double norm = found ? __longlong_as_double(0x7ff0000000000000ll) : sqrt(sumsq);
+        const bool clipped = !found && clip > 0.0f && norm > (double)clip;
+        mpt_check_result r;
+        r.found_inf = found ? 1 : 0;
+        r.clipped = clipped ? 1 : 0;
+        r.grad_norm = norm;
+        r.clip_coef = clipped ? __double2float_rn((double)clip / norm) : 1.0f;
+        r.reserved = 0;
+        r.n_nonfinite = nnf;
+        *out = r;
+        c->nonfinite_acc = 0;
+        c->ticket = 0;
+    }
+}
+
+extern "C" int mpt_check_flat_noalloc(const void* d_grads_half, int64_t n, float scale,
+                                      float clip, mpt_check_result* d_result,
+                                      void* cuda_stream)
+{
+    if (!d_grads_half || !d_result || n <= 0 ||
+        (reinterpret_cast<uintptr_t>(d_grads_half) & 1) != 0 ||
+        (reinterpret_cast<uintptr_t>(d_result) & 7) != 0)
+        return MPT_ERR_INVALID_ARG;
+    if (!finite(scale) || !(scale > 0.0f) || !finite(clip))
+        return MPT_ERR_INVALID_ARG;
+    if (n > MPT_NOALLOC_MAX_ELEMS)
+        return MPT_ERR_TOO_LARGE;
+
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess) {
+        cudaGetLastError();
+        return MPT_ERR_CUDA;
+    }
+    if (dev < 0 || dev >= kNoAllocMaxDevices)
+        return MPT_ERR_CUDA;
+    // In host code the array's name is a host-side stand-in, not a device
+    // address: look the address up once per device, with that device current.
+    std::call_once(g_noalloc_once[dev], [dev] {
+        g_noalloc_status[dev] =
+            cudaGetSymbolAddress(reinterpret_cast<void**>(&g_noalloc_addr[dev]), g_noalloc_scratch);
+    });
+    if (g_noalloc_status[dev] != cudaSuccess || !g_noalloc_addr[dev])
+        return MPT_ERR_CUDA;
+    unsigned char* scratch = g_noalloc_addr[dev];
+
+    cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
+    // the counters must start at zero whatever the previous call left
+    if (cudaMemsetAsync(scratch, 0, kNoAllocCtrlBytes, st) != cudaSuccess) {
+        cudaGetLastError();
+        return MPT_ERR_CUDA;
+    }
+    const float inv_scale = 1.0f / scale;
+    int e2 = 0;
+    const bool pow2 = std::frexp(scale, &e2) == 0.5f && (e2 - 1) >= -15 && (e2 - 1) <= 100;
+    const double dscale = pow2 ? std::ldexp(1.0, 1008 - (e2 - 1)) : 0.0;
+    const unsigned int bins = (unsigned int)((n + kNoAllocChunk - 1) / kNoAllocChunk);
+    const uint16_t* g = static_cast<const uint16_t*>(d_grads_half);
+    if (pow2)
+        check_flat_kernel<true><<<bins, kThreads, 0, st>>>(g, n, scratch, d_result, inv_scale, dscale, clip);
+    else
+        check_flat_kernel<false><<<bins, kThreads, 0, st>>>(g, n, scratch, d_result, inv_scale, dscale, clip);
+    if (cudaGetLastError() != cudaSuccess)
+        return MPT_ERR_CUDA;
+    return MPT_OK;
+}
