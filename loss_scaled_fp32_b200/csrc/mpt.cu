@@ -72,7 +72,8 @@ mpt_config defaults()
 
 // Arena offsets (16-element aligned) and the work bins: every tensor larger
 // than kSmallTensor is cut into chunk-sized ranges, one bin each; the small
-// tensors are packed, in list order, into bins of at most `chunk` elements.
+// tensors are packed, in list order, into bins of at most kPackedMaxElems
+// elements and kMaxPackedSegs tensors.
 int build_layout(const int64_t* sizes, int32_t n, int32_t chunk, Layout& L)
 {
     L.arena_off.resize(n);
@@ -89,18 +90,13 @@ int build_layout(const int64_t* sizes, int32_t n, int32_t chunk, Layout& L)
         if (sizes[i] <= kSmallTensor)
             continue;
         for (int64_t c = 0; c < sizes[i]; c += chunk) {
-            Seg s{};
-            s.tensor_begin = c;
-            s.arena_begin = L.arena_off[i] + c;
-            s.tensor = i;
-            s.len = (int32_t)std::min<int64_t>(chunk, sizes[i] - c);
-            s.local_begin = 0;
             Bin b{};
-            b.first_seg = (int32_t)L.segs.size();
-            b.n_segs = 1;
-            b.n_elems = s.len;
+            b.tensor_begin = c;
+            b.arena_begin = L.arena_off[i] + c;
+            b.tensor = i;
+            b.n_elems = (int32_t)std::min<int64_t>(chunk, sizes[i] - c);
+            b.n_segs = 0;
             b.kind = kChunkBin;
-            L.segs.push_back(s);
             L.bins.push_back(b);
         }
     }
@@ -110,13 +106,13 @@ int build_layout(const int64_t* sizes, int32_t n, int32_t chunk, Layout& L)
         if (sizes[i] > kSmallTensor)
             continue;
         const int32_t len = (int32_t)sizes[i];
-        if (have_open && (open.n_elems + len > chunk || open.n_segs == kMaxPackedSegs)) {
+        if (have_open && (open.n_elems + len > kPackedMaxElems || open.n_segs == kMaxPackedSegs)) {
             L.bins.push_back(open);
             have_open = false;
         }
         if (!have_open) {
             open = Bin{};
-            open.first_seg = (int32_t)L.segs.size();
+            open.tensor = (int32_t)L.segs.size();
             open.kind = kPackedBin;
             have_open = true;
         }

@@ -13,28 +13,34 @@ constexpr int kDefaultChunk = 32768;       // elements per work bin
 constexpr int kChunkQuantum = 2048;        // chunk sizes are multiples of this
 constexpr int kMaxChunk = 1 << 20;
 constexpr int kSmallTensor = 1024;         // tensors up to this size are packed
-constexpr int kMaxPackedSegs = 1024;       // tensors per packed bin
+constexpr int kPackedMaxElems = 4096;      // elements per packed bin
+constexpr int kMaxPackedSegs = 256;        // tensors per packed bin
+constexpr int kPackedUnroll = kPackedMaxElems / kThreads;  // elements per thread
 
 enum BinKind : int32_t {
     kChunkBin = 0,   // one contiguous range of one tensor (vectorised)
     kPackedBin = 1,  // several whole small tensors (flattened, scalar)
 };
 
-// One contiguous range of one tensor.
+// One whole small tensor inside a packed bin.
 struct __align__(16) Seg {
-    int64_t tensor_begin;  // first element, counted inside the tensor
+    int64_t tensor_begin;  // first element, counted inside the tensor (0)
     int64_t arena_begin;   // the same element's index in the three arenas
     int32_t tensor;        // index into the gradient-pointer table
     int32_t len;           // elements
-    int32_t local_begin;   // offset of this range inside its bin
+    int32_t local_begin;   // offset of this tensor inside its bin
     int32_t pad;
 };
 
-// The work of one CTA.
+// The work of one CTA.  A chunk bin carries its range inline (one dependent
+// load less before the first gradient load); a packed bin points at n_segs
+// consecutive Seg entries.
 struct __align__(16) Bin {
-    int32_t first_seg;
-    int32_t n_segs;
-    int32_t n_elems;
+    int64_t tensor_begin;  // chunk bin: first element of the range in its tensor
+    int64_t arena_begin;   // chunk bin: that element's index in the arenas
+    int32_t tensor;        // chunk bin: tensor index; packed bin: first Seg index
+    int32_t n_elems;       // elements in the bin
+    int32_t n_segs;        // packed bin: number of tensors; chunk bin: 0
     int32_t kind;
 };
 

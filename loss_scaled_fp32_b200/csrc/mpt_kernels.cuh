@@ -61,31 +61,33 @@ struct UpdateArgs {
 // small helpers
 // ---------------------------------------------------------------------------
 
-__device__ __forceinline__ bool seg_ok(const Seg& s, const Tables& t)
+__device__ __forceinline__ bool range_ok(int32_t tensor, int64_t tensor_begin, int64_t arena_begin,
+                                         int64_t len, const Tables& t)
 {
-    if (s.tensor < 0 || s.tensor >= t.ntensors || s.len < 0 || s.tensor_begin < 0)
+    if (tensor < 0 || tensor >= t.ntensors || len < 0 || tensor_begin < 0)
         return false;
-    const TensorInfo ti = t.tensors[s.tensor];
-    return s.tensor_begin + s.len <= ti.size && s.arena_begin == ti.arena_off + s.tensor_begin &&
-           s.arena_begin + s.len <= t.arena_total;
+    const TensorInfo ti = t.tensors[tensor];
+    return tensor_begin + len <= ti.size && arena_begin == ti.arena_off + tensor_begin &&
+           arena_begin + len <= t.arena_total;
 }
 
-// Checked mode: validate a bin and all of its ranges before touching memory.
+// Checked mode: validate a bin (and every tensor of a packed bin) before any
+// gradient, master or momentum address is formed from it.
 __device__ __forceinline__ bool bin_ok(const Bin& bin, const Tables& t)
 {
-    if (bin.first_seg < 0 || bin.n_segs < 1 || bin.n_segs > kMaxPackedSegs ||
-        bin.first_seg + bin.n_segs > t.nsegs || bin.n_elems < 0)
+    if (bin.n_elems < 0)
         return false;
-    if (bin.kind == kChunkBin) {
-        const Seg s = t.segs[bin.first_seg];
-        return bin.n_segs == 1 && s.len == bin.n_elems && s.local_begin == 0 && seg_ok(s, t);
-    }
-    if (bin.kind != kPackedBin)
+    if (bin.kind == kChunkBin)
+        return bin.n_segs == 0 &&
+               range_ok(bin.tensor, bin.tensor_begin, bin.arena_begin, bin.n_elems, t);
+    if (bin.kind != kPackedBin || bin.tensor < 0 || bin.n_segs < 1 ||
+        bin.n_segs > kMaxPackedSegs || bin.n_elems > kPackedMaxElems ||
+        bin.tensor + bin.n_segs > t.nsegs)
         return false;
     int32_t expect = 0;
     for (int k = 0; k < bin.n_segs; ++k) {
-        const Seg s = t.segs[bin.first_seg + k];
-        if (s.local_begin != expect || !seg_ok(s, t))
+        const Seg s = t.segs[bin.tensor + k];
+        if (s.local_begin != expect || !range_ok(s.tensor, s.tensor_begin, s.arena_begin, s.len, t))
             return false;
         expect += s.len;
     }
@@ -268,23 +270,40 @@ __device__ __forceinline__ unsigned int block_sum_u32(unsigned int x, unsigned i
     return t;
 }
 
-// Exact count of non-finite elements of a bin (run only by a CTA that saw one).
-__device__ unsigned int count_nonfinite(const Bin& bin, const Tables& t)
+// Exact count of non-finite elements in n gradients (run only by a CTA that
+// saw one).
+__device__ __forceinline__ unsigned int count_nonfinite(const uint16_t* g, int n)
 {
     unsigned int c = 0;
-    for (int k = 0; k < bin.n_segs; ++k) {
-        const Seg s = t.segs[bin.first_seg + k];
-        const uint16_t* g = t.grads[s.tensor] + s.tensor_begin;
-        for (int j = threadIdx.x; j < s.len; j += kThreads)
-            c += ((g[j] & 0x7C00u) == 0x7C00u) ? 1u : 0u;
-    }
+    for (int j = threadIdx.x; j < n; j += kThreads)
+        c += ((g[j] & 0x7C00u) == 0x7C00u) ? 1u : 0u;
     return c;
+}
+
+// Packed bins: the gradient pointer and offset of each tensor are staged in
+// shared memory once, then every thread handles kPackedUnroll elements with
+// all of its loads issued before any is used.
+struct PackedStage {
+    int32_t begin[kMaxPackedSegs];
+    const uint16_t* gptr[kMaxPackedSegs];
+    int64_t arena[kMaxPackedSegs];
+};
+
+__device__ __forceinline__ void stage_packed(const Bin& bin, const Tables& t, PackedStage& st)
+{
+    for (int k = threadIdx.x; k < bin.n_segs; k += kThreads) {
+        const Seg s = t.segs[bin.tensor + k];
+        st.begin[k] = s.local_begin;
+        st.gptr[k] = t.grads[s.tensor] + s.tensor_begin;
+        st.arena[k] = s.arena_begin;
+    }
+    __syncthreads();
 }
 
 template <bool kPow2, bool kChecked>
 __global__ void __launch_bounds__(kThreads) check_kernel(CheckArgs a)
 {
-    __shared__ int32_t s_begin[kMaxPackedSegs];
+    __shared__ PackedStage st;
     __shared__ double s_red[kWarps];
     __shared__ unsigned int s_ured[kWarps];
     __shared__ int s_last;
@@ -296,25 +315,43 @@ __global__ void __launch_bounds__(kThreads) check_kernel(CheckArgs a)
     if constexpr (kChecked)
         valid = bin_ok(bin, t);
 
+    const uint16_t* chunk_g = nullptr;
     if (valid) {
         if (bin.kind == kChunkBin) {
-            const Seg sg = t.segs[bin.first_seg];
-            check_range<kPow2>(t.grads[sg.tensor] + sg.tensor_begin, sg.len, a, s);
+            chunk_g = t.grads[bin.tensor] + bin.tensor_begin;
+            check_range<kPow2>(chunk_g, bin.n_elems, a, s);
         } else {
-            for (int k = threadIdx.x; k < bin.n_segs; k += kThreads)
-                s_begin[k] = t.segs[bin.first_seg + k].local_begin;
-            __syncthreads();
-            for (int j = threadIdx.x; j < bin.n_elems; j += kThreads) {
-                const Seg sg = t.segs[bin.first_seg + find_seg(s_begin, bin.n_segs, j)];
-                sq_half<kPow2>(__ldg(t.grads[sg.tensor] + sg.tensor_begin + (j - sg.local_begin)), a, s);
+            stage_packed(bin, t, st);
+            uint16_t h[kPackedUnroll];
+#pragma unroll
+            for (int i = 0; i < kPackedUnroll; ++i) {
+                const int j = threadIdx.x + i * kThreads;
+                h[i] = 0;  // +0: adds nothing, is finite
+                if (j < bin.n_elems) {
+                    const int k = find_seg(st.begin, bin.n_segs, j);
+                    h[i] = __ldg(st.gptr[k] + (j - st.begin[k]));
+                }
             }
+#pragma unroll
+            for (int i = 0; i < kPackedUnroll; ++i)
+                sq_half<kPow2>(h[i], a, s);
         }
     }
 
     // Non-finite count: exact, but only computed by a CTA that saw one.
     unsigned int nf = 0;
-    if (__syncthreads_or((s.nf & 0x80008000u) != 0))
-        nf = block_sum_u32(count_nonfinite(bin, t), s_ured);
+    if (__syncthreads_or((s.nf & 0x80008000u) != 0)) {
+        unsigned int c = 0;
+        if (bin.kind == kChunkBin) {
+            c = count_nonfinite(chunk_g, bin.n_elems);
+        } else {
+            for (int j = threadIdx.x; j < bin.n_elems; j += kThreads) {
+                const int k = find_seg(st.begin, bin.n_segs, j);
+                c += ((st.gptr[k][j - st.begin[k]] & 0x7C00u) == 0x7C00u) ? 1u : 0u;
+            }
+        }
+        nf = block_sum_u32(c, s_ured);
+    }
 
     const double part = block_sum(s.a0 + s.a1, s_red);
     if (threadIdx.x == 0) {
@@ -520,7 +557,7 @@ __device__ __forceinline__ void count_range(const uint16_t* g, int len, uint32_t
 template <bool kStale, bool kChecked>
 __global__ void __launch_bounds__(kThreads) update_kernel(UpdateArgs a)
 {
-    __shared__ int32_t s_begin[kMaxPackedSegs];
+    __shared__ PackedStage st;
     __shared__ unsigned int s_ured[kWarps];
 
     const Tables& t = a.t;
@@ -539,25 +576,47 @@ __global__ void __launch_bounds__(kThreads) update_kernel(UpdateArgs a)
 
     if (valid) {
         if (bin.kind == kChunkBin) {
-            const Seg sg = t.segs[bin.first_seg];
-            const uint16_t* g = t.grads[sg.tensor] + sg.tensor_begin;
+            const uint16_t* g = t.grads[bin.tensor] + bin.tensor_begin;
             if (skip)
-                count_range(g, sg.len, nz2, ns2);
+                count_range(g, bin.n_elems, nz2, ns2);
             else
-                update_range<kStale>(g, a.master + sg.arena_begin, a.momentum + sg.arena_begin,
-                                     a.w16 + sg.arena_begin, sg.len, p, nz2, ns2, stale);
+                update_range<kStale>(g, a.master + bin.arena_begin, a.momentum + bin.arena_begin,
+                                     a.w16 + bin.arena_begin, bin.n_elems, p, nz2, ns2, stale);
         } else {
-            for (int k = threadIdx.x; k < bin.n_segs; k += kThreads)
-                s_begin[k] = t.segs[bin.first_seg + k].local_begin;
-            __syncthreads();
-            for (int j = threadIdx.x; j < bin.n_elems; j += kThreads) {
-                const Seg sg = t.segs[bin.first_seg + find_seg(s_begin, bin.n_segs, j)];
-                const int64_t off = j - sg.local_begin;
-                const uint16_t gh = __ldcs(t.grads[sg.tensor] + sg.tensor_begin + off);
-                count_half(gh, nz2, ns2);
-                if (!skip) {
-                    const int64_t e = sg.arena_begin + off;
-                    upd_scalar<kStale>(gh, a.master + e, a.momentum + e, a.w16 + e, p, stale);
+            stage_packed(bin, t, st);
+            constexpr int kU = 4;
+            for (int base = 0; base < bin.n_elems; base += kU * kThreads) {
+                uint16_t gh[kU];
+                int64_t e[kU];
+                float w[kU], v[kU];
+#pragma unroll
+                for (int i = 0; i < kU; ++i) {
+                    const int j = base + threadIdx.x + i * kThreads;
+                    e[i] = -1;
+                    if (j < bin.n_elems) {
+                        const int k = find_seg(st.begin, bin.n_segs, j);
+                        const int off = j - st.begin[k];
+                        gh[i] = __ldcs(st.gptr[k] + off);
+                        e[i] = st.arena[k] + off;
+                        if (!skip) {
+                            w[i] = __ldcs(a.master + e[i]);
+                            v[i] = __ldcs(a.momentum + e[i]);
+                        }
+                    }
+                }
+#pragma unroll
+                for (int i = 0; i < kU; ++i) {
+                    if (e[i] < 0)
+                        continue;
+                    count_half(gh[i], nz2, ns2);
+                    if (!skip) {
+                        const float w0 = w[i];
+                        upd1(__half2float(__ushort_as_half(gh[i])), w[i], v[i], p);
+                        __stcs(a.master + e[i], w[i]);
+                        __stcs(a.momentum + e[i], v[i]);
+                        a.w16[e[i]] = __half_as_ushort(__float2half_rn(w[i]));
+                        stale1<kStale>(w0, w[i], stale);
+                    }
                 }
             }
         }
@@ -565,16 +624,16 @@ __global__ void __launch_bounds__(kThreads) update_kernel(UpdateArgs a)
 
     const unsigned int nz = block_sum_u32((nz2 & 0xFFFFu) + (nz2 >> 16), s_ured);
     const unsigned int ns = block_sum_u32((ns2 & 0xFFFFu) + (ns2 >> 16), s_ured);
-    unsigned int st = 0;
+    unsigned int n_stale = 0;
     if constexpr (kStale)
-        st = block_sum_u32(stale, s_ured);
+        n_stale = block_sum_u32(stale, s_ured);
     if (threadIdx.x == 0) {
         Ctrl* cw = a.ctrl;
         if (valid) {
             atomicAdd(&cw->zero_acc, (unsigned long long)(bin.n_elems - nz));
             atomicAdd(&cw->subnormal_acc, (unsigned long long)(nz - ns));
-            if (st)
-                atomicAdd(&cw->stale_acc, (unsigned long long)st);
+            if (n_stale)
+                atomicAdd(&cw->stale_acc, (unsigned long long)n_stale);
         } else {
             atomicOr(&cw->error, (unsigned int)kErrBadBin);
         }

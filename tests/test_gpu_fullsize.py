@@ -1,0 +1,154 @@
+"""GPU parity at the workloads' full sizes, in the launch configuration the
+benchmark times (default chunking, one mpt_step call per step).
+
+The whole step runs on the GPU over every parameter.  The oracle checks it
+the way its definition allows at any size:
+  * pass 1 of the oracle (overflow flag, range counts, sum of squares) runs
+    over the FULL gradient list every step -> found_inf, the counts, the new S
+    and the clean-step counter exact, the norm within 1e-5 relative;
+  * pass 2 (the per-element update) runs on a sample of elements -- random
+    positions plus the first and last element of every tensor -- whose FP32
+    master, FP32 momentum and FP16 copy the oracle carries from step to step;
+    they must match the GPU's bit for bit (whenever the two clip
+    coefficients agree, which they do unless two summation orders of the
+    binary64 norm straddle a binary32 rounding boundary).
+The loss scale evolves as in training: each step's gradients are drawn at the
+S the previous step returned, so overflow, backoff and growth happen
+naturally (plus each workload's injected inf/NaN steps).
+"""
+import math
+import os
+from concurrent.futures import ThreadPoolExecutor
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads as W
+from loss_scaled_fp32_b200 import MPT, Config
+
+pytestmark = pytest.mark.gpu
+
+THREADS = min(16, os.cpu_count() or 1)
+
+
+class Sampled:
+    def __init__(self, cfg, n_random=200_000, seed=0):
+        self.cfg = cfg
+        sizes = np.array(cfg.sizes, dtype=np.int64)
+        starts = np.concatenate([[0], np.cumsum(sizes)[:-1]])
+        rng = np.random.default_rng(seed)
+        idx = rng.integers(0, cfg.n_params, n_random)
+        idx = np.unique(np.concatenate([idx, starts, starts + sizes - 1]))
+        self.tensor = np.searchsorted(starts, idx, side="right") - 1
+        self.elem = idx - starts[self.tensor]
+        self.layout = W.GradLayout(cfg.sizes)
+        self.opt = MPT(cfg.sizes, Config(backoff=cfg.backoff, growth=cfg.growth,
+                                         growth_interval=cfg.growth_interval))
+        for i, m in enumerate(W.make_master(cfg, "cuda")):
+            self.opt.master(i).copy_(m)
+        self.opt.refresh_half()
+        self.opt.set_scaler_state(cfg.scale0, 0)
+        # flat arena views through the tensor views' addresses
+        base = self.opt.master(0).data_ptr()
+        arena_off = np.array([(self.opt.master(i).data_ptr() - base) // 4
+                              for i in range(len(cfg.sizes))], dtype=np.int64)
+        self.arena_idx = torch.from_numpy(arena_off[self.tensor] + self.elem).cuda()
+        total = int(arena_off[-1] + sizes[-1])
+        self.m_flat = self.opt.master(0).view(-1).as_strided((total,), (1,))
+        self.v_flat = self.opt.momentum(0).view(-1).as_strided((total,), (1,))
+        self.h_flat = self.opt.w16(0).view(-1).as_strided((total,), (1,))
+        m, v, h = self.gather()
+        assert np.array_equal(h, oracle.rne16(m))
+        self.w, self.v, self.h = m, v, h
+        self.grad_idx = torch.from_numpy(np.array(self.layout.offsets)[self.tensor] + self.elem).cuda()
+        self.ocfg = oracle.scaler_cfg(backoff=cfg.backoff, growth=cfg.growth,
+                                      growth_interval=cfg.growth_interval)
+        self.scale = cfg.scale0
+        self.clean = 0
+        self.flat = torch.zeros(self.layout.total, dtype=torch.int16, device="cuda")
+        self.views = self.layout.views(self.flat)
+        self.host = torch.empty(self.layout.total, dtype=torch.int16, pin_memory=True)
+
+    def gather(self):
+        m = self.m_flat.index_select(0, self.arena_idx).cpu().numpy()
+        v = self.v_flat.index_select(0, self.arena_idx).cpu().numpy()
+        h = self.h_flat.index_select(0, self.arena_idx).cpu().numpy().view(np.uint16)
+        return m, v, h
+
+    def full_check(self, scale):
+        """Oracle pass 1 over every tensor (threads over groups of tensors; the
+        binary64 partials are added in list order)."""
+        hv = [v.numpy().view(np.uint16) for v in self.layout.views(self.host)]
+        groups = np.array_split(np.arange(len(hv)), min(THREADS, len(hv)))
+        res = list(ThreadPoolExecutor(THREADS).map(
+            lambda g: oracle.check([hv[i] for i in g], scale), groups))
+        total = res[0]
+        for r in res[1:]:
+            total.found_inf |= r.found_inf
+            total.n_zero += r.n_zero
+            total.n_subnormal += r.n_subnormal
+            total.n_nonfinite += r.n_nonfinite
+            total.sumsq += r.sumsq
+        return total
+
+    def step(self, k):
+        cfg = self.cfg
+        W.make_grads(cfg, k, self.scale, self.layout, "cuda", out=self.flat)
+        self.host.copy_(self.flat)
+        r = self.opt.step(self.views, self.scale, cfg.lr, cfg.momentum, cfg.weight_decay,
+                          cfg.clip)
+        ro = oracle.clip_coef(self.full_check(self.scale), cfg.clip)
+        for key in ("found_inf", "clipped", "n_zero", "n_subnormal", "n_nonfinite"):
+            assert r[key] == getattr(ro, key), (k, key, r[key], getattr(ro, key))
+        new_scale, self.clean = oracle.scaler_next(self.ocfg, ro.found_inf, self.scale, self.clean)
+        assert r["new_scale"] == new_scale and r["clean_run"] == self.clean, k
+        if ro.found_inf:
+            assert math.isinf(r["grad_norm"])
+        else:
+            assert abs(r["grad_norm"] - ro.norm) <= 1e-5 * ro.norm
+            g16 = self.flat.index_select(0, self.grad_idx).cpu().numpy().view(np.uint16)
+            oracle.update(g16, self.w, self.v, self.h, self.scale, ro.clipped, ro.clip_coef,
+                          cfg.lr, cfg.momentum, cfg.weight_decay)
+        m, v, h = self.gather()
+        if r["clip_coef"] == ro.clip_coef:
+            assert m.tobytes() == self.w.tobytes(), k
+            assert v.tobytes() == self.v.tobytes(), k
+            assert h.tobytes() == self.h.tobytes(), k
+        else:  # one-ulp coefficient difference at a rounding boundary
+            from parity import ulp_diff_f16, ulp_diff_f32
+            assert ulp_diff_f32(m, self.w).max() <= 1 and ulp_diff_f32(v, self.v).max() <= 1
+            assert ulp_diff_f16(h, self.h).max() <= 1
+            self.w, self.v, self.h = m, v, h
+        self.scale = r["new_scale"]
+        return r
+
+
+def run(name, steps=None):
+    cfg = W.get(name)
+    s = Sampled(cfg)
+    out = [s.step(k) for k in range(1, (steps or cfg.steps) + 1)]
+    s.opt.close()
+    return out
+
+
+def test_fullsize_resnet50():
+    rs = run("resnet50")
+    assert all(r["found_inf"] == 0 for r in rs)
+
+
+def test_fullsize_gpt2_medium_dynamic_scale_and_clip():
+    rs = run("gpt2_medium")
+    assert any(r["found_inf"] for r in rs)           # S grows until it overflows
+    assert any(r["clipped"] for r in rs)
+
+
+def test_fullsize_gpt_1p3b():
+    rs = run("gpt_1p3b")
+    assert all(r["found_inf"] == 0 for r in rs)
+
+
+def test_fullsize_ragged20k():
+    rs = run("ragged20k")
+    assert sum(r["found_inf"] for r in rs) >= 20      # 20 injected + natural overflow
