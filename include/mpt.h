@@ -95,7 +95,7 @@ typedef struct {
 } mpt_step_result;
 
 typedef struct {
-    uint64_t steps;           /* mpt_step calls that completed                  */
+    uint64_t steps;           /* steps completed on the device                  */
     uint64_t skipped;         /* of which were skipped on overflow              */
     float scale;              /* current S (last new_scale, or the value set)   */
     int32_t clean_run;        /* current clean-step counter                     */
@@ -147,31 +147,62 @@ int mpt_tensor_views(const mpt_handle* h, int32_t i, float** master,
  * Errors: MPT_ERR_INVALID_ARG, MPT_ERR_CUDA, MPT_ERR_BROKEN. */
 int mpt_refresh_half(mpt_handle* h, void* cuda_stream);
 
+/* The loss-scale state (S and the clean-step counter) lives in the
+ * workspace and is advanced on the device by every step, so steps can be
+ * queued without the host waiting; the handle keeps a host mirror that every
+ * waiting call (mpt_step, mpt_wait, mpt_set_scaler_state) refreshes. */
+
 /* One optimizer step.  d_grads_half is a HOST array of n DEVICE pointers, the
  * FP16 (binary16) gradients of the n tensors, computed from a loss multiplied
  * by `scale` (any 2-byte alignment; contents are only read).  lr, momentum
  * and weight_decay are eta, mu and lambda; clip <= 0 disables clipping.
  * Work is queued on cuda_stream and the call waits for it (it reads the
- * result back), then updates the handle's scale state: out->new_scale is
- * the S to pass to the next step.  On overflow the arenas are untouched.
- * Errors: MPT_ERR_INVALID_ARG, MPT_ERR_CUDA, MPT_ERR_DEVICE_CHECK,
- * MPT_ERR_BROKEN; on any error *out is not written and the scale state does
- * not change. */
+ * 112-byte control block back).  The scale state advances from `scale`:
+ * out->new_scale is the S for the next step.  On overflow the arenas are
+ * untouched.  Errors: MPT_ERR_INVALID_ARG, MPT_ERR_CUDA,
+ * MPT_ERR_DEVICE_CHECK (checked mode; the bins that passed their check were
+ * updated), MPT_ERR_BROKEN; on an argument error nothing is queued. */
 int mpt_step(mpt_handle* h, const void* const* d_grads_half, float scale,
              float lr, float momentum, float weight_decay, float clip,
              void* cuda_stream, mpt_step_result* out);
 
-/* Counters and the last result.  Errors: MPT_ERR_INVALID_ARG. */
+/* The same step, queued on cuda_stream without waiting: S is the device
+ * scale state (see mpt_device_scale), the gradients must have been computed
+ * from a loss multiplied by that device value, and the step advances the
+ * state on the device.  Nothing is read back; call mpt_wait for the result
+ * of the last queued step.  The gradient buffers must stay unchanged until
+ * the queued work has run.  Errors: MPT_ERR_INVALID_ARG, MPT_ERR_CUDA,
+ * MPT_ERR_BROKEN. */
+int mpt_step_async(mpt_handle* h, const void* const* d_grads_half, float lr,
+                   float momentum, float weight_decay, float clip, void* cuda_stream);
+
+/* Wait for the work queued on cuda_stream and return the result of the last
+ * step (out may be NULL); refreshes the host mirror of the scale state and
+ * the counters.  Errors: MPT_ERR_INVALID_ARG, MPT_ERR_CUDA,
+ * MPT_ERR_DEVICE_CHECK, MPT_ERR_BROKEN. */
+int mpt_wait(mpt_handle* h, void* cuda_stream, mpt_step_result* out);
+
+/* Device address of the binary32 loss scale S that the next
+ * mpt_step_async uses (inside the workspace): a training loop multiplies its
+ * loss by it on the device.  Errors: MPT_ERR_INVALID_ARG. */
+int mpt_device_scale(const mpt_handle* h, float** d_scale);
+
+/* Counters and the last result, as of the last waiting call.
+ * Errors: MPT_ERR_INVALID_ARG. */
 int mpt_stats(const mpt_handle* h, mpt_stats_t* out);
 
-/* Read / set the loss-scale state (checkpoint and resume).  set requires a
- * finite scale > 0 and clean_run >= 0.  Errors: MPT_ERR_INVALID_ARG. */
+/* Read the host mirror of the loss-scale state (as of the last waiting
+ * call) / set the state on the device and the host (checkpoint and resume;
+ * synchronous, call it with no step in flight).  set requires a finite
+ * scale > 0 and clean_run >= 0.  Errors: MPT_ERR_INVALID_ARG, MPT_ERR_CUDA,
+ * MPT_ERR_BROKEN. */
 int mpt_get_scaler_state(const mpt_handle* h, float* scale, int32_t* clean_run);
 int mpt_set_scaler_state(mpt_handle* h, float scale, int32_t clean_run);
 
 /* Time both kernels of every following step with CUDA events recorded on the
- * step's stream (summed into mpt_stats_t); enable = 0 turns it off.
- * Errors: MPT_ERR_INVALID_ARG, MPT_ERR_CUDA. */
+ * step's stream (summed into mpt_stats_t at the next waiting call, or when
+ * 256 timed steps are pending); enable = 0 turns it off (and waits for the
+ * pending events).  Errors: MPT_ERR_INVALID_ARG, MPT_ERR_CUDA. */
 int mpt_set_timing(mpt_handle* h, int32_t enable);
 
 /* Release the handle's host resources.  The workspace is the caller's and is

@@ -115,6 +115,9 @@ def lib():
             "mpt_set_timing": [vp, i32],
             "mpt_destroy": [vp],
             "mpt_check_flat_noalloc": [vp, ctypes.c_int64, f32, f32, vp, vp],
+            "mpt_step_async": [vp, vp, f32, f32, f32, f32, vp],
+            "mpt_wait": [vp, vp, ctypes.POINTER(StepResult)],
+            "mpt_device_scale": [vp, ctypes.POINTER(vp)],
         }
         for name, args in sig.items():
             fn = getattr(L, name)
@@ -212,21 +215,44 @@ class MPT:
     def step(self, grads, scale, lr, momentum, weight_decay, clip=0.0, stream=None):
         """``grads``: list of FP16 (or int16 bit-pattern) CUDA tensors, or an
         array from :func:`grad_pointers`.  Returns the step result as a dict."""
-        if isinstance(grads, ctypes.Array):
-            ptrs = grads
-        else:
-            if len(grads) != self.n:
-                raise ValueError(f"expected {self.n} gradient tensors, got {len(grads)}")
-            for g, n in zip(grads, self.sizes):
-                if g.numel() != n or g.element_size() != 2 or g.device != self.device:
-                    raise ValueError("gradient tensor does not match its size/dtype/device")
-                if not g.is_contiguous():
-                    raise ValueError("gradient tensors must be contiguous")
-            ptrs = grad_pointers(grads)
+        ptrs = self._ptrs(grads)
         r = StepResult()
         _check(lib().mpt_step(self._h, ptrs, scale, lr, momentum, weight_decay, clip,
                               _stream_ptr(stream, self.device), ctypes.byref(r)), "mpt_step")
         return r.as_dict()
+
+    def _ptrs(self, grads):
+        if isinstance(grads, ctypes.Array):
+            return grads
+        if len(grads) != self.n:
+            raise ValueError(f"expected {self.n} gradient tensors, got {len(grads)}")
+        for g, n in zip(grads, self.sizes):
+            if g.numel() != n or g.element_size() != 2 or g.device != self.device:
+                raise ValueError("gradient tensor does not match its size/dtype/device")
+            if not g.is_contiguous():
+                raise ValueError("gradient tensors must be contiguous")
+        return grad_pointers(grads)
+
+    def step_async(self, grads, lr, momentum, weight_decay, clip=0.0, stream=None):
+        """Queue one step without waiting; S is the device scale state
+        (:meth:`device_scale`).  Call :meth:`wait` for the result."""
+        _check(lib().mpt_step_async(self._h, self._ptrs(grads), lr, momentum, weight_decay, clip,
+                                    _stream_ptr(stream, self.device)), "mpt_step_async")
+
+    def wait(self, stream=None):
+        """Wait for the queued steps; returns the last step's result."""
+        r = StepResult()
+        _check(lib().mpt_wait(self._h, _stream_ptr(stream, self.device), ctypes.byref(r)),
+               "mpt_wait")
+        return r.as_dict()
+
+    def device_scale(self):
+        """A 1-element float32 CUDA tensor aliasing the device scale state."""
+        p = ctypes.c_void_p()
+        _check(lib().mpt_device_scale(self._h, ctypes.byref(p)), "mpt_device_scale")
+        off = p.value - self.workspace.data_ptr()
+        import torch
+        return self.workspace[off:off + 4].view(torch.float32)
 
     def stats(self):
         s = Stats()

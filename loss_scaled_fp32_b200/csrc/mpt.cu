@@ -1,18 +1,20 @@
 // mpt.cu -- host side of libmpt: the C ABI declared in include/mpt.h.
 //
-// One step = two kernel launches on the caller's stream and one 80-byte
-// read-back of the control block:
+// One step = two kernel launches on the caller's stream and, for the
+// waiting call, one 112-byte read-back of the control block:
 //   check_kernel  (2 B/param)  overflow flag, range counts, sum of squares,
 //                              last-CTA finish -> norm, clip coefficient
 //   update_kernel (20 B/param) fused unscale/clip/decay/momentum/master/FP16,
 //                              or counting only when the step overflowed
 // The launch order alone carries the check result to the update, so no host
-// decision sits between the two kernels.  The loss-scale state machine runs on
-// the host once the result is back.
+// decision sits between the two kernels.  The loss-scale state machine runs in
+// the check kernel's last CTA and keeps S on the device, so that steps can be
+// queued without waiting (mpt_step_async); the host mirrors it on read-back.
 #include <cuda_runtime.h>
 
 #include <cmath>
 #include <cstdlib>
+#include <cstddef>
 #include <cstring>
 #include <mutex>
 #include <new>
@@ -24,7 +26,7 @@
 
 using namespace mpt;
 
-static_assert(sizeof(Ctrl) == 80, "the control block read back each step is 80 bytes");
+static_assert(sizeof(Ctrl) == 112, "the control block read back each step is 112 bytes");
 
 namespace {
 
@@ -154,6 +156,8 @@ bool finite(float x) { return std::isfinite(x); }
 
 }  // namespace
 
+constexpr int kTimingRing = 256;  // steps whose kernel events may be pending
+
 struct mpt_handle {
     int device = 0;
     int32_t n = 0;
@@ -174,22 +178,27 @@ struct mpt_handle {
     std::vector<const void*> last_ptrs;
     bool ptrs_uploaded = false;
     const void** pinned_ptrs = nullptr;  // staging of the pointer table
+    cudaEvent_t ptrs_copied = nullptr;   // the last pointer-table copy is done
     Ctrl* mailbox = nullptr;             // pinned copy of the control block
-    float scale = 1.0f;
+    float scale = 1.0f;                  // host mirror of the device scale state
     int32_t clean_run = 0;
     mpt_stats_t stats{};
     bool broken = false;
+    // kernel timing: ring of (start, between, end) events, one per step
     bool timing = false;
-    cudaEvent_t ev[3] = {nullptr, nullptr, nullptr};
+    std::vector<cudaEvent_t> tev;
+    int64_t t_head = 0, t_tail = 0;
 };
 
 static void release(mpt_handle* h)
 {
     if (!h)
         return;
-    for (cudaEvent_t& e : h->ev)
+    for (cudaEvent_t e : h->tev)
         if (e)
             cudaEventDestroy(e);
+    if (h->ptrs_copied)
+        cudaEventDestroy(h->ptrs_copied);
     if (h->pinned_ptrs)
         cudaFreeHost(h->pinned_ptrs);
     if (h->mailbox)
@@ -197,34 +206,190 @@ static void release(mpt_handle* h)
     delete h;
 }
 
-// Loss-scale state machine (dynamic loss scaling): back off on overflow,
-// grow after growth_interval consecutive clean steps.
-static float next_scale(const mpt_config& c, bool found_inf, float scale, int32_t& clean)
+// Add the durations of the oldest timed step (waits for its last event).
+static bool timing_pop(mpt_handle* h)
 {
-    if (found_inf) {
-        clean = 0;
-        const float s = scale * c.backoff;
-        return s < c.min_scale ? c.min_scale : s;
-    }
-    clean += 1;
-    if (c.growth_interval > 0 && clean >= c.growth_interval) {
-        clean = 0;
-        const float s = scale * c.growth;
-        return s > c.max_scale ? c.max_scale : s;
-    }
-    return scale;
+    const int slot = (int)(h->t_tail % kTimingRing);
+    cudaEvent_t* e = &h->tev[3 * slot];
+    float t01 = 0.0f, t12 = 0.0f;
+    if (cudaEventSynchronize(e[2]) != cudaSuccess ||
+        cudaEventElapsedTime(&t01, e[0], e[1]) != cudaSuccess ||
+        cudaEventElapsedTime(&t12, e[1], e[2]) != cudaSuccess)
+        return false;
+    h->stats.check_ms_total += t01;
+    h->stats.update_ms_total += t12;
+    h->stats.timed_steps += 1;
+    h->t_tail += 1;
+    return true;
 }
 
-template <bool kPow2, bool kChecked>
+template <bool kChecked>
 static void launch_check(const CheckArgs& a, cudaStream_t st)
 {
-    check_kernel<kPow2, kChecked><<<a.t.nbins, kThreads, 0, st>>>(a);
+    check_kernel<kChecked><<<a.t.nbins, kThreads, 0, st>>>(a);
 }
 
+// The update kernel may start while the check kernel drains (programmatic
+// dependent launch): its CTAs take the SMs the check CTAs free, load their
+// work descriptors, then wait for the check result (griddepcontrol.wait).
 template <bool kStale, bool kChecked>
 static void launch_update(const UpdateArgs& a, cudaStream_t st)
 {
-    update_kernel<kStale, kChecked><<<a.t.nbins, kThreads, 0, st>>>(a);
+    cudaLaunchConfig_t lc = {};
+    lc.gridDim = dim3((unsigned int)a.t.nbins);
+    lc.blockDim = dim3(kThreads);
+    lc.dynamicSmemBytes = 0;
+    lc.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    lc.attrs = attr;
+    lc.numAttrs = 1;
+    cudaLaunchKernelEx(&lc, update_kernel<kStale, kChecked>, a);
+}
+
+// Queue one step (both kernels) on st.  scale_on_device: S comes from the
+// device scale state instead of host_scale.
+static int enqueue_step(mpt_handle* h, const void* const* d_grads_half, bool scale_on_device,
+                        float host_scale, float lr, float momentum, float weight_decay,
+                        float clip, cudaStream_t st)
+{
+    for (int32_t i = 0; i < h->n; ++i) {
+        const uintptr_t p = reinterpret_cast<uintptr_t>(d_grads_half[i]);
+        if (p == 0 || (p & 1))
+            return MPT_ERR_INVALID_ARG;
+    }
+    const size_t ptr_bytes = sizeof(void*) * (size_t)h->n;
+
+    // The pointer table crosses to the device only when it changed; the
+    // staging buffer is reused only once its previous copy has completed.
+    if (!h->ptrs_uploaded || std::memcmp(h->last_ptrs.data(), d_grads_half, ptr_bytes) != 0) {
+        if (h->ptrs_uploaded && cudaEventSynchronize(h->ptrs_copied) != cudaSuccess)
+            return MPT_ERR_CUDA;
+        std::memcpy(h->pinned_ptrs, d_grads_half, ptr_bytes);
+        if (cudaMemcpyAsync(h->d_ptrs, h->pinned_ptrs, ptr_bytes, cudaMemcpyHostToDevice, st) != cudaSuccess ||
+            cudaEventRecord(h->ptrs_copied, st) != cudaSuccess)
+            return MPT_ERR_CUDA;
+        std::memcpy(h->last_ptrs.data(), d_grads_half, ptr_bytes);
+        h->ptrs_uploaded = true;
+    }
+
+    Tables t;
+    t.bins = h->d_bins;
+    t.segs = h->d_segs;
+    t.tensors = h->d_tinfo;
+    t.grads = h->d_ptrs;
+    t.nbins = (int32_t)h->L.bins.size();
+    t.nsegs = (int32_t)h->L.segs.size();
+    t.ntensors = h->n;
+    t.pad = 0;
+    t.arena_total = h->L.arena_total;
+
+    CheckArgs ca;
+    ca.t = t;
+    ca.partials = h->d_partials;
+    ca.ctrl = h->d_ctrl;
+    ca.host_scale = host_scale;
+    ca.scale_on_device = scale_on_device ? 1 : 0;
+    ca.clip = clip;
+    ca.scaler.backoff = h->cfg.backoff;
+    ca.scaler.growth = h->cfg.growth;
+    ca.scaler.growth_interval = h->cfg.growth_interval;
+    ca.scaler.min_scale = h->cfg.min_scale;
+    ca.scaler.max_scale = h->cfg.max_scale;
+
+    UpdateArgs ua;
+    ua.t = t;
+    ua.master = h->d_master;
+    ua.momentum = h->d_momentum;
+    ua.w16 = h->d_w16;
+    ua.ctrl = h->d_ctrl;
+    ua.lr = lr;
+    ua.mu = momentum;
+    ua.wd = weight_decay;
+
+    cudaEvent_t* ev = nullptr;
+    if (h->timing) {
+        if (h->t_head - h->t_tail == kTimingRing && !timing_pop(h))
+            return MPT_ERR_CUDA;
+        ev = &h->tev[3 * (int)(h->t_head % kTimingRing)];
+        h->t_head += 1;
+    }
+    const bool checked = (h->cfg.flags & MPT_FLAG_CHECKED) != 0;
+    const bool stale = (h->cfg.flags & MPT_FLAG_COUNT_STALE) != 0;
+    bool ok = true;
+    if (ev)
+        ok = ok && cudaEventRecord(ev[0], st) == cudaSuccess;
+    checked ? launch_check<true>(ca, st) : launch_check<false>(ca, st);
+    if (ev)
+        ok = ok && cudaEventRecord(ev[1], st) == cudaSuccess;
+    if (stale)
+        checked ? launch_update<true, true>(ua, st) : launch_update<true, false>(ua, st);
+    else
+        checked ? launch_update<false, true>(ua, st) : launch_update<false, false>(ua, st);
+    if (ev)
+        ok = ok && cudaEventRecord(ev[2], st) == cudaSuccess;
+    ok = ok && cudaGetLastError() == cudaSuccess;
+    return ok ? MPT_OK : MPT_ERR_CUDA;
+}
+
+// Read the control block back (waits for the stream), mirror the device
+// state on the host and turn it into a step result.
+static int read_result(mpt_handle* h, cudaStream_t st, mpt_step_result* out)
+{
+    if (cudaMemcpyAsync(h->mailbox, h->d_ctrl, sizeof(Ctrl), cudaMemcpyDeviceToHost, st) != cudaSuccess ||
+        cudaStreamSynchronize(st) != cudaSuccess)
+        return MPT_ERR_CUDA;
+    while (h->t_tail < h->t_head)
+        if (!timing_pop(h))
+            return MPT_ERR_CUDA;
+    const Ctrl& c = *h->mailbox;
+    if (c.error != 0)
+        return MPT_ERR_DEVICE_CHECK;
+    const bool stale = (h->cfg.flags & MPT_FLAG_COUNT_STALE) != 0;
+    mpt_step_result r{};
+    r.found_inf = c.found_inf;
+    r.clipped = c.clipped;
+    r.grad_norm = c.norm;
+    r.clip_coef = c.coef;
+    r.n_zero = c.zero_acc;
+    r.n_subnormal = c.subnormal_acc;
+    r.n_nonfinite = c.n_nonfinite;
+    r.n_fp16_stale = stale ? c.stale_acc : 0;
+    r.new_scale = c.scale;
+    r.clean_run = c.clean_run;
+    h->scale = c.scale;
+    h->clean_run = c.clean_run;
+    if (c.steps_total > h->stats.steps)
+        h->stats.n_fp16_stale_total += r.n_fp16_stale;
+    h->stats.steps = c.steps_total;
+    h->stats.skipped = c.skipped_total;
+    h->stats.scale = h->scale;
+    h->stats.clean_run = h->clean_run;
+    h->stats.last = r;
+    if (out)
+        *out = r;
+    return MPT_OK;
+}
+
+static int fail_cuda(mpt_handle* h)
+{
+    cudaGetLastError();
+    h->broken = true;
+    h->ptrs_uploaded = false;
+    return MPT_ERR_CUDA;
+}
+
+static bool upload_scaler_state(mpt_handle* h, float scale, int32_t clean_run)
+{
+    struct {
+        float scale;
+        int32_t clean_run;
+    } v{scale, clean_run};
+    static_assert(offsetof(Ctrl, clean_run) == offsetof(Ctrl, scale) + sizeof(float),
+                  "scale and clean_run are adjacent");
+    return cudaMemcpy(reinterpret_cast<char*>(h->d_ctrl) + offsetof(Ctrl, scale), &v, sizeof v,
+                      cudaMemcpyHostToDevice) == cudaSuccess;
 }
 
 extern "C" {
@@ -314,6 +479,8 @@ int mpt_create(const int64_t* sizes, int32_t n, const mpt_config* cfg, void* d_w
               cudaMemset(ws + L.off_master, 0, L.total - L.off_master) == cudaSuccess &&
               cudaHostAlloc(reinterpret_cast<void**>(&h->pinned_ptrs), sizeof(void*) * n, cudaHostAllocDefault) == cudaSuccess &&
               cudaHostAlloc(reinterpret_cast<void**>(&h->mailbox), sizeof(Ctrl), cudaHostAllocDefault) == cudaSuccess &&
+              cudaEventCreateWithFlags(&h->ptrs_copied, cudaEventDisableTiming) == cudaSuccess &&
+              upload_scaler_state(h, 1.0f, 0) &&
               cudaDeviceSynchronize() == cudaSuccess;
     if (!ok) {
         cudaGetLastError();
@@ -369,119 +536,45 @@ int mpt_step(mpt_handle* h, const void* const* d_grads_half, float scale, float 
     if (!finite(scale) || !(scale > 0.0f) || !finite(lr) || !finite(momentum) ||
         !finite(weight_decay) || !finite(clip))
         return MPT_ERR_INVALID_ARG;
-    for (int32_t i = 0; i < h->n; ++i) {
-        const uintptr_t p = reinterpret_cast<uintptr_t>(d_grads_half[i]);
-        if (p == 0 || (p & 1))
-            return MPT_ERR_INVALID_ARG;
-    }
     cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
-    const size_t ptr_bytes = sizeof(void*) * (size_t)h->n;
+    int rc = enqueue_step(h, d_grads_half, false, scale, lr, momentum, weight_decay, clip, st);
+    if (rc == MPT_ERR_CUDA)
+        return fail_cuda(h);
+    if (rc != MPT_OK)
+        return rc;
+    rc = read_result(h, st, out);
+    return rc == MPT_ERR_CUDA ? fail_cuda(h) : rc;
+}
 
-    // The pointer table crosses to the device only when it changed.
-    if (!h->ptrs_uploaded || std::memcmp(h->last_ptrs.data(), d_grads_half, ptr_bytes) != 0) {
-        std::memcpy(h->pinned_ptrs, d_grads_half, ptr_bytes);
-        if (cudaMemcpyAsync(h->d_ptrs, h->pinned_ptrs, ptr_bytes, cudaMemcpyHostToDevice, st) != cudaSuccess) {
-            h->broken = true;
-            return MPT_ERR_CUDA;
-        }
-        std::memcpy(h->last_ptrs.data(), d_grads_half, ptr_bytes);
-        h->ptrs_uploaded = true;
-    }
+int mpt_step_async(mpt_handle* h, const void* const* d_grads_half, float lr, float momentum,
+                   float weight_decay, float clip, void* cuda_stream)
+{
+    if (!h || !d_grads_half)
+        return MPT_ERR_INVALID_ARG;
+    if (h->broken)
+        return MPT_ERR_BROKEN;
+    if (!finite(lr) || !finite(momentum) || !finite(weight_decay) || !finite(clip))
+        return MPT_ERR_INVALID_ARG;
+    const int rc = enqueue_step(h, d_grads_half, true, 0.0f, lr, momentum, weight_decay, clip,
+                                static_cast<cudaStream_t>(cuda_stream));
+    return rc == MPT_ERR_CUDA ? fail_cuda(h) : rc;
+}
 
-    Tables t;
-    t.bins = h->d_bins;
-    t.segs = h->d_segs;
-    t.tensors = h->d_tinfo;
-    t.grads = h->d_ptrs;
-    t.nbins = (int32_t)h->L.bins.size();
-    t.nsegs = (int32_t)h->L.segs.size();
-    t.ntensors = h->n;
-    t.pad = 0;
-    t.arena_total = h->L.arena_total;
+int mpt_wait(mpt_handle* h, void* cuda_stream, mpt_step_result* out)
+{
+    if (!h)
+        return MPT_ERR_INVALID_ARG;
+    if (h->broken)
+        return MPT_ERR_BROKEN;
+    const int rc = read_result(h, static_cast<cudaStream_t>(cuda_stream), out);
+    return rc == MPT_ERR_CUDA ? fail_cuda(h) : rc;
+}
 
-    CheckArgs ca;
-    ca.t = t;
-    ca.partials = h->d_partials;
-    ca.ctrl = h->d_ctrl;
-    ca.inv_scale = 1.0f / scale;
-    ca.clip = clip;
-    int e2 = 0;
-    const bool pow2 = std::frexp(scale, &e2) == 0.5f && (e2 - 1) >= -15 && (e2 - 1) <= 100;
-    ca.dscale = pow2 ? std::ldexp(1.0, 1008 - (e2 - 1)) : 0.0;
-
-    UpdateArgs ua;
-    ua.t = t;
-    ua.master = h->d_master;
-    ua.momentum = h->d_momentum;
-    ua.w16 = h->d_w16;
-    ua.ctrl = h->d_ctrl;
-    ua.inv_scale = ca.inv_scale;
-    ua.lr = lr;
-    ua.mu = momentum;
-    ua.wd = weight_decay;
-
-    const bool checked = (h->cfg.flags & MPT_FLAG_CHECKED) != 0;
-    const bool stale = (h->cfg.flags & MPT_FLAG_COUNT_STALE) != 0;
-    bool ok = true;
-    if (h->timing)
-        ok = ok && cudaEventRecord(h->ev[0], st) == cudaSuccess;
-    if (pow2)
-        checked ? launch_check<true, true>(ca, st) : launch_check<true, false>(ca, st);
-    else
-        checked ? launch_check<false, true>(ca, st) : launch_check<false, false>(ca, st);
-    if (h->timing)
-        ok = ok && cudaEventRecord(h->ev[1], st) == cudaSuccess;
-    if (stale)
-        checked ? launch_update<true, true>(ua, st) : launch_update<true, false>(ua, st);
-    else
-        checked ? launch_update<false, true>(ua, st) : launch_update<false, false>(ua, st);
-    if (h->timing)
-        ok = ok && cudaEventRecord(h->ev[2], st) == cudaSuccess;
-    ok = ok && cudaGetLastError() == cudaSuccess;
-    ok = ok && cudaMemcpyAsync(h->mailbox, h->d_ctrl, sizeof(Ctrl), cudaMemcpyDeviceToHost, st) == cudaSuccess;
-    ok = ok && cudaStreamSynchronize(st) == cudaSuccess;
-    if (!ok) {
-        cudaGetLastError();
-        h->broken = true;
-        h->ptrs_uploaded = false;
-        return MPT_ERR_CUDA;
-    }
-    if (h->timing) {
-        float t01 = 0.0f, t12 = 0.0f;
-        if (cudaEventElapsedTime(&t01, h->ev[0], h->ev[1]) == cudaSuccess &&
-            cudaEventElapsedTime(&t12, h->ev[1], h->ev[2]) == cudaSuccess) {
-            h->stats.check_ms_total += t01;
-            h->stats.update_ms_total += t12;
-            h->stats.timed_steps += 1;
-        }
-    }
-
-    const Ctrl& c = *h->mailbox;
-    if (c.error != 0)
-        return MPT_ERR_DEVICE_CHECK;
-
-    mpt_step_result r{};
-    r.found_inf = c.found_inf;
-    r.clipped = c.clipped;
-    r.grad_norm = c.norm;
-    r.clip_coef = c.coef;
-    r.n_zero = c.zero_acc;
-    r.n_subnormal = c.subnormal_acc;
-    r.n_nonfinite = c.n_nonfinite;
-    r.n_fp16_stale = stale ? c.stale_acc : 0;
-    int32_t clean = h->clean_run;
-    r.new_scale = next_scale(h->cfg, c.found_inf != 0, scale, clean);
-    r.clean_run = clean;
-
-    h->scale = r.new_scale;
-    h->clean_run = clean;
-    h->stats.steps += 1;
-    h->stats.skipped += c.found_inf ? 1 : 0;
-    h->stats.scale = h->scale;
-    h->stats.clean_run = clean;
-    h->stats.last = r;
-    h->stats.n_fp16_stale_total += r.n_fp16_stale;
-    *out = r;
+int mpt_device_scale(const mpt_handle* h, float** d_scale)
+{
+    if (!h || !d_scale)
+        return MPT_ERR_INVALID_ARG;
+    *d_scale = &h->d_ctrl->scale;
     return MPT_OK;
 }
 
@@ -506,6 +599,10 @@ int mpt_set_scaler_state(mpt_handle* h, float scale, int32_t clean_run)
 {
     if (!h || !finite(scale) || !(scale > 0.0f) || clean_run < 0)
         return MPT_ERR_INVALID_ARG;
+    if (h->broken)
+        return MPT_ERR_BROKEN;
+    if (!upload_scaler_state(h, scale, clean_run))
+        return fail_cuda(h);
     h->scale = scale;
     h->clean_run = clean_run;
     h->stats.scale = scale;
@@ -517,13 +614,19 @@ int mpt_set_timing(mpt_handle* h, int32_t enable)
 {
     if (!h)
         return MPT_ERR_INVALID_ARG;
-    if (enable && !h->ev[0]) {
-        for (cudaEvent_t& e : h->ev) {
+    if (enable && h->tev.empty()) {
+        h->tev.assign(3 * kTimingRing, nullptr);
+        for (cudaEvent_t& e : h->tev) {
             if (cudaEventCreate(&e) != cudaSuccess) {
                 cudaGetLastError();
                 return MPT_ERR_CUDA;
             }
         }
+    }
+    if (!enable) {
+        while (h->t_tail < h->t_head)
+            if (!timing_pop(h))
+                return fail_cuda(h);
     }
     h->timing = enable != 0;
     return MPT_OK;
@@ -601,15 +704,15 @@ check_flat_kernel(const uint16_t* g, int64_t n, unsigned char* scratch, mpt_chec
     const int64_t begin = (int64_t)blockIdx.x * kNoAllocChunk;
     const int len = (int)(n - begin < kNoAllocChunk ? n - begin : kNoAllocChunk);
 
-    CheckArgs a{};
+    SqParams a{};
     a.inv_scale = inv_scale;
     a.dscale = dscale;
-    a.clip = clip;
+    a.pow2 = kPow2;
     SqAcc s;
     check_range<kPow2>(g + begin, len, a, s);
 
     unsigned int nf = 0;
-    if (__syncthreads_or((s.nf & 0x80008000u) != 0)) {
+    if (__syncthreads_or(s.saw_nonfinite())) {
         unsigned int cnt = 0;
         for (int j = threadIdx.x; j < len; j += kThreads)
             cnt += ((g[begin + j] & 0x7C00u) == 0x7C00u) ? 1u : 0u;

@@ -70,6 +70,13 @@ struct __align__(16) Ctrl {
     int32_t clipped;
     float coef;
     unsigned int error;    // checked-mode error bits of both kernels
+    float inv_scale;       // binary32 1/S of this step (read by the update)
+    float scale_used;      // S of this step
+    // loss-scale state, advanced by the check kernel's last CTA
+    float scale;           // S for the next step
+    int32_t clean_run;     // consecutive clean steps so far
+    unsigned long long steps_total;
+    unsigned long long skipped_total;
 };
 
 enum ErrorBits : unsigned int {

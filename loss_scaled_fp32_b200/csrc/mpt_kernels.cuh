@@ -36,13 +36,23 @@ struct Tables {
     int64_t arena_total;
 };
 
+// Loss-scale state machine parameters (dynamic loss scaling).
+struct ScalerParams {
+    float backoff;
+    float growth;
+    int32_t growth_interval;
+    float min_scale;
+    float max_scale;
+};
+
 struct CheckArgs {
     Tables t;
-    double* partials;  // one binary64 partial sum of squares per bin
+    double* partials;     // one binary64 partial sum of squares per bin
     Ctrl* ctrl;
-    float inv_scale;   // binary32 1/S
-    float clip;        // <= 0: off
-    double dscale;     // power-of-two S only: 2^1008 / S (see sq_bits)
+    float host_scale;     // S the gradients carry, when given by the host
+    int32_t scale_on_device;  // 1: S is ctrl->scale (asynchronous steps)
+    float clip;           // <= 0: off
+    ScalerParams scaler;
 };
 
 struct UpdateArgs {
@@ -50,12 +60,31 @@ struct UpdateArgs {
     float* master;
     float* momentum;
     uint16_t* w16;
-    Ctrl* ctrl;
-    float inv_scale;
+    Ctrl* ctrl;           // check result: skip flag, clip coefficient, 1/S
     float lr;
     float mu;
     float wd;
 };
+
+// What the squares need from S: the binary32 reciprocal 1/S and, when S is a
+// power of two 2^e with -15 <= e <= 100, the binary64 constant 2^(1008-e).
+struct SqParams {
+    float inv_scale;
+    double dscale;
+    bool pow2;
+};
+
+__device__ __forceinline__ SqParams sq_params(float S)
+{
+    SqParams q;
+    q.inv_scale = __fdiv_rn(1.0f, S);
+    const uint32_t b = __float_as_uint(S);
+    const int biased = (int)((b >> 23) & 0xFFu);
+    const int e = biased - 127;
+    q.pow2 = (b & 0x807FFFFFu) == 0 && biased != 0 && e >= -15 && e <= 100;
+    q.dscale = q.pow2 ? __longlong_as_double((long long)(1008 - e + 1023) << 52) : 0.0;
+    return q;
+}
 
 // ---------------------------------------------------------------------------
 // small helpers
@@ -121,6 +150,8 @@ __device__ __forceinline__ uint32_t h2_bits(__half2 h)
 struct SqAcc {
     double a0 = 0.0, a1 = 0.0;
     uint32_t nf = 0;  // bit 15 or 31 set <=> some element seen was +-inf/NaN
+
+    __device__ __forceinline__ bool saw_nonfinite() const { return (nf & 0x80008000u) != 0; }
 };
 
 // Square of one unscaled gradient, accumulated in binary64.
@@ -136,7 +167,7 @@ struct SqAcc {
 //
 // Other S: x is rounded to binary32 first, as the definition says.
 template <bool kPow2>
-__device__ __forceinline__ void sq_bits(uint32_t mag_hi_word, uint16_t h, const CheckArgs& a,
+__device__ __forceinline__ void sq_bits(uint32_t mag_hi_word, uint16_t h, const SqParams& a,
                                         double& acc)
 {
     if constexpr (kPow2) {
@@ -149,7 +180,7 @@ __device__ __forceinline__ void sq_bits(uint32_t mag_hi_word, uint16_t h, const 
 }
 
 template <bool kPow2>
-__device__ __forceinline__ void sq_word(uint32_t w, const CheckArgs& a, SqAcc& s)
+__device__ __forceinline__ void sq_word(uint32_t w, const SqParams& a, SqAcc& s)
 {
     sq_bits<kPow2>((w << 10) & 0x01FFFC00u, (uint16_t)(w & 0xFFFFu), a, s.a0);
     sq_bits<kPow2>((w >> 6) & 0x01FFFC00u, (uint16_t)(w >> 16), a, s.a1);
@@ -161,14 +192,14 @@ __device__ __forceinline__ void sq_word(uint32_t w, const CheckArgs& a, SqAcc& s
 }
 
 template <bool kPow2>
-__device__ __forceinline__ void sq_half(uint16_t h, const CheckArgs& a, SqAcc& s)
+__device__ __forceinline__ void sq_half(uint16_t h, const SqParams& a, SqAcc& s)
 {
     sq_bits<kPow2>(((uint32_t)h << 10) & 0x01FFFC00u, h, a, s.a0);
     s.nf |= (~(uint32_t)h & 0x7C00u) - 0x0400u;
 }
 
 template <bool kPow2>
-__device__ __forceinline__ void sq_vec(uint4 v, const CheckArgs& a, SqAcc& s)
+__device__ __forceinline__ void sq_vec(uint4 v, const SqParams& a, SqAcc& s)
 {
     sq_word<kPow2>(v.x, a, s);
     sq_word<kPow2>(v.y, a, s);
@@ -177,7 +208,7 @@ __device__ __forceinline__ void sq_vec(uint4 v, const CheckArgs& a, SqAcc& s)
 }
 
 template <bool kPow2>
-__device__ __forceinline__ void sq_vec(uint2 v, const CheckArgs& a, SqAcc& s)
+__device__ __forceinline__ void sq_vec(uint2 v, const SqParams& a, SqAcc& s)
 {
     sq_word<kPow2>(v.x, a, s);
     sq_word<kPow2>(v.y, a, s);
@@ -186,7 +217,7 @@ __device__ __forceinline__ void sq_vec(uint2 v, const CheckArgs& a, SqAcc& s)
 // One contiguous range: 16-B loads when aligned, 8-B when 8-B aligned, else
 // 2-B loads; unrolled so that every thread has 64 B of loads in flight.
 template <bool kPow2, typename Vec>
-__device__ __forceinline__ void check_range_vec(const uint16_t* g, int len, const CheckArgs& a,
+__device__ __forceinline__ void check_range_vec(const uint16_t* g, int len, const SqParams& a,
                                                 SqAcc& s)
 {
     constexpr int kPer = sizeof(Vec) / 2;
@@ -210,7 +241,7 @@ __device__ __forceinline__ void check_range_vec(const uint16_t* g, int len, cons
 }
 
 template <bool kPow2>
-__device__ __forceinline__ void check_range(const uint16_t* g, int len, const CheckArgs& a,
+__device__ __forceinline__ void check_range(const uint16_t* g, int len, const SqParams& a,
                                             SqAcc& s)
 {
     const uintptr_t p = reinterpret_cast<uintptr_t>(g);
@@ -300,16 +331,26 @@ __device__ __forceinline__ void stage_packed(const Bin& bin, const Tables& t, Pa
     __syncthreads();
 }
 
-template <bool kPow2, bool kChecked>
-__global__ void __launch_bounds__(kThreads) check_kernel(CheckArgs a)
+template <bool kChecked>
+__global__ void __launch_bounds__(kThreads, 8) check_kernel(CheckArgs a)
 {
     __shared__ PackedStage st;
     __shared__ double s_red[kWarps];
     __shared__ unsigned int s_ured[kWarps];
     __shared__ int s_last;
 
+    // Let the update kernel (launched with programmatic stream serialization)
+    // be scheduled as soon as every CTA of this grid is running; it waits for
+    // this grid's completion before it reads the result.
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+
     const Tables& t = a.t;
     const Bin bin = t.bins[blockIdx.x];
+    // S of these gradients: the host's, or the device state the previous
+    // step left (it changes only in this kernel's last CTA, after every other
+    // CTA has finished reading it)
+    const float S = a.scale_on_device ? a.ctrl->scale : a.host_scale;
+    const SqParams q = sq_params(S);
     SqAcc s;
     bool valid = true;
     if constexpr (kChecked)
@@ -319,28 +360,40 @@ __global__ void __launch_bounds__(kThreads) check_kernel(CheckArgs a)
     if (valid) {
         if (bin.kind == kChunkBin) {
             chunk_g = t.grads[bin.tensor] + bin.tensor_begin;
-            check_range<kPow2>(chunk_g, bin.n_elems, a, s);
+            if (q.pow2)
+                check_range<true>(chunk_g, bin.n_elems, q, s);
+            else
+                check_range<false>(chunk_g, bin.n_elems, q, s);
         } else {
             stage_packed(bin, t, st);
-            uint16_t h[kPackedUnroll];
+            constexpr int kU = 8;
+            for (int base = 0; base < bin.n_elems; base += kU * kThreads) {
+                uint16_t h[kU];
 #pragma unroll
-            for (int i = 0; i < kPackedUnroll; ++i) {
-                const int j = threadIdx.x + i * kThreads;
-                h[i] = 0;  // +0: adds nothing, is finite
-                if (j < bin.n_elems) {
-                    const int k = find_seg(st.begin, bin.n_segs, j);
-                    h[i] = __ldg(st.gptr[k] + (j - st.begin[k]));
+                for (int i = 0; i < kU; ++i) {
+                    const int j = base + threadIdx.x + i * kThreads;
+                    h[i] = 0;  // +0: adds nothing, is finite
+                    if (j < bin.n_elems) {
+                        const int k = find_seg(st.begin, bin.n_segs, j);
+                        h[i] = __ldg(st.gptr[k] + (j - st.begin[k]));
+                    }
+                }
+                if (q.pow2) {
+#pragma unroll
+                    for (int i = 0; i < kU; ++i)
+                        sq_half<true>(h[i], q, s);
+                } else {
+#pragma unroll
+                    for (int i = 0; i < kU; ++i)
+                        sq_half<false>(h[i], q, s);
                 }
             }
-#pragma unroll
-            for (int i = 0; i < kPackedUnroll; ++i)
-                sq_half<kPow2>(h[i], a, s);
         }
     }
 
     // Non-finite count: exact, but only computed by a CTA that saw one.
     unsigned int nf = 0;
-    if (__syncthreads_or((s.nf & 0x80008000u) != 0)) {
+    if (__syncthreads_or(s.saw_nonfinite())) {
         unsigned int c = 0;
         if (bin.kind == kChunkBin) {
             c = count_nonfinite(chunk_g, bin.n_elems);
@@ -388,7 +441,28 @@ __global__ void __launch_bounds__(kThreads) check_kernel(CheckArgs a)
         c->found_inf = found ? 1 : 0;
         c->clipped = clipped ? 1 : 0;
         c->coef = clipped ? __double2float_rn((double)a.clip / norm) : 1.0f;
+        c->inv_scale = q.inv_scale;
+        c->scale_used = S;
         c->error = err;
+        // Loss-scale state machine: on overflow skip and multiply S by beta;
+        // after growth_interval consecutive clean steps multiply S by alpha.
+        const ScalerParams& sp = a.scaler;
+        int32_t clean = c->clean_run;
+        float next = S;
+        if (found) {
+            next = fmaxf(__fmul_rn(S, sp.backoff), sp.min_scale);
+            clean = 0;
+            c->skipped_total += 1;
+        } else {
+            clean += 1;
+            if (sp.growth_interval > 0 && clean >= sp.growth_interval) {
+                next = fminf(__fmul_rn(S, sp.growth), sp.max_scale);
+                clean = 0;
+            }
+        }
+        c->scale = next;
+        c->clean_run = clean;
+        c->steps_total += 1;
         c->nonfinite_acc = 0;
         c->error_acc = 0;
         c->zero_acc = 0;
@@ -569,9 +643,12 @@ __global__ void __launch_bounds__(kThreads) update_kernel(UpdateArgs a)
     if constexpr (kChecked)
         valid = bin_ok(bin, t);
 
+    // Wait until the check kernel has finished and its result is visible
+    // (returns at once when this grid was launched without overlap).
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     const Ctrl* c = a.ctrl;
     const bool skip = c->found_inf != 0;
-    const UpdParams p{a.inv_scale, c->coef, a.lr, a.mu, a.wd};
+    const UpdParams p{c->inv_scale, c->coef, a.lr, a.mu, a.wd};
     uint32_t nz2 = 0, ns2 = 0, stale = 0;
 
     if (valid) {

@@ -210,3 +210,51 @@ def test_stats_and_timing():
     assert st["steps"] == 3 and st["timed_steps"] == 3
     assert st["check_ms_total"] > 0 and st["update_ms_total"] > 0
     assert st["scale"] == p.scale
+
+
+# ---------------------------------------------------------------------------
+# queued (asynchronous) steps with the loss scale kept on the device
+# ---------------------------------------------------------------------------
+
+def test_async_steps_follow_the_oracle():
+    """Steps queued back to back with mpt_step_async: S is read from and
+    advanced on the device; each step's gradients are drawn at the S the
+    oracle's state machine predicts, so the device must agree with it."""
+    plan = {3: [(1, 7, 0x7C00)], 8: [(0, 0, 0x7E00)]}
+    cfg = custom([60_000, 1031, 5, 40_000], law=("log2_uniform", -26.0, -2.0), scale0=2.0 ** 12,
+                 growth_interval=2, clip=0.3, steps=10, injections=lambda s: plan.get(s, []))
+    p = Pair(cfg)
+    ocfg, S, clean = p.ocfg, cfg.scale0, 0
+    bufs = []
+    for k in range(1, cfg.steps + 1):
+        host = p.grads(k, S)
+        dev = host.cuda()
+        bufs.append(dev)                       # must outlive the queued step
+        p.opt.step_async(p.layout.views(dev), cfg.lr, cfg.momentum, cfg.weight_decay, cfg.clip)
+        hv = [v.numpy().view(np.uint16) for v in p.layout.views(host)]
+        ro = oracle.step(p.state, hv, S, cfg.lr, cfg.momentum, cfg.weight_decay, clip=cfg.clip,
+                         cfg=ocfg)
+        S = ro["new_scale"]
+    r = p.opt.wait()
+    assert r["new_scale"] == S and p.opt.scaler_state() == (S, p.state.clean_run)
+    assert p.opt.device_scale().item() == S
+    st = p.opt.stats()
+    assert st["steps"] == cfg.steps and st["skipped"] == 2
+    p.compare_state("after queued steps", exact=True)
+
+
+def test_sync_and_async_steps_share_the_scale_state():
+    cfg = custom([30_000], scale0=2.0 ** 8, growth_interval=1, steps=4)
+    p = Pair(cfg)
+    r, _ = p.step()                            # S = 2^8 given by the host
+    assert r["new_scale"] == 2.0 ** 9
+    assert p.opt.device_scale().item() == 2.0 ** 9
+    host = p.grads(2, 2.0 ** 9)
+    dev = host.cuda()
+    p.opt.step_async(p.layout.views(dev), cfg.lr, cfg.momentum, cfg.weight_decay)
+    hv = [v.numpy().view(np.uint16) for v in p.layout.views(host)]
+    oracle.step(p.state, hv, 2.0 ** 9, cfg.lr, cfg.momentum, cfg.weight_decay, cfg=p.ocfg)
+    assert p.opt.wait()["new_scale"] == 2.0 ** 10
+    p.compare_state("mixed", exact=True)
+    p.opt.set_scaler_state(3.0, 0)             # any S, also not a power of two
+    assert p.opt.device_scale().item() == 3.0
