@@ -40,10 +40,13 @@ class _Result(ctypes.Structure):
                 ("clip_coef", ctypes.c_float), ("n_zero", ctypes.c_uint64),
                 ("n_subnormal", ctypes.c_uint64), ("n_nonfinite", ctypes.c_uint64),
                 ("n_stale", ctypes.c_uint64), ("new_scale", ctypes.c_float),
-                ("new_clean_run", ctypes.c_int32)]
+                ("new_clean_run", ctypes.c_int32), ("max_mag16", ctypes.c_uint16),
+                ("max_abs", ctypes.c_float), ("exp_hist", ctypes.c_uint64 * 32)]
 
     def as_dict(self):
-        return {name: getattr(self, name) for name, _ in self._fields_}
+        d = {name: getattr(self, name) for name, _ in self._fields_}
+        d["exp_hist"] = list(self.exp_hist)
+        return d
 
 
 def lib():
@@ -72,6 +75,8 @@ def lib():
                                ctypes.POINTER(ScalerCfg), ctypes.POINTER(ctypes.c_int32),
                                u32, ctypes.POINTER(_Result)]
         L.orc_step.restype = None
+        L.orc_direct_scale.argtypes = [f32, f32, f32, f32]
+        L.orc_direct_scale.restype = f32
         _LIB = L
     return _LIB
 
@@ -154,6 +159,11 @@ def update(g16, w, v, w16, scale, clipped, coef, lr, momentum, weight_decay, fla
     inv = np.float32(1.0) / np.float32(scale)
     return lib().orc_update(g16.size, _ptr(g16), _ptr(w), _ptr(v), _ptr(w16), inv,
                             int(clipped), coef, lr, momentum, weight_decay, flags)
+
+
+def direct_scale(max_abs, margin=2.0, min_scale=2.0 ** -24, max_scale=2.0 ** 24):
+    """S = 65504 / (margin * max|g|) (binary64, rounded to binary32, clamped)."""
+    return lib().orc_direct_scale(max_abs, margin, min_scale, max_scale)
 
 
 def scaler_next(cfg, found_inf, scale, clean_run):

@@ -126,12 +126,15 @@ void orc_check(const uint16_t* const* grads, const int64_t* sizes, int32_t n,
 {
     int32_t found = 0;
     uint64_t nz = 0, ns = 0, nf = 0;
+    uint16_t max_mag = 0;
     double sumsq = 0.0;
 
+    memset(r->exp_hist, 0, sizeof r->exp_hist);
     for (int32_t i = 0; i < n; ++i) {
         for (int64_t j = 0; j < sizes[i]; ++j) {
             uint16_t h = grads[i][j];
             uint16_t mag = (uint16_t)(h & 0x7fffu);
+            r->exp_hist[mag >> 10] += 1;   /* binade of the scaled gradient */
             /* Step 6, "Overflow detection": any +-inf or NaN (exponent field
              * all ones) anywhere in the list. */
             if (mag >= 0x7c00u) {
@@ -143,6 +146,8 @@ void orc_check(const uint16_t* const* grads, const int64_t* sizes, int32_t n,
                 nz += 1;
             else if (mag < 0x0400u)
                 ns += 1;
+            if (mag > max_mag)   /* bit patterns of magnitudes order like values */
+                max_mag = mag;
             /* Global L2 norm of the unscaled gradients: every square of a
              * binary32 value is exact in binary64; the sum is binary64. */
             double x = (double)unscale(h, inv_scale);
@@ -154,6 +159,8 @@ void orc_check(const uint16_t* const* grads, const int64_t* sizes, int32_t n,
     r->n_subnormal = ns;
     r->n_nonfinite = nf;
     r->sumsq = sumsq;
+    r->max_mag16 = max_mag;
+    r->max_abs = unscale(max_mag, inv_scale);
 }
 
 void orc_clip_coef(orc_result* r, float clip)
@@ -225,6 +232,20 @@ float orc_scaler_next(const orc_scaler_cfg* cfg, int32_t found_inf, float scale,
         return s > cfg->max_scale ? cfg->max_scale : s;
     }
     return scale;
+}
+
+float orc_direct_scale(float max_abs, float margin, float min_scale, float max_scale)
+{
+    if (!(max_abs > 0.0f))
+        return 0.0f;
+    /* 65504 is the largest binary16 value; the margin leaves headroom for
+     * the next step's gradients to be larger than this one's. */
+    float s = (float)(65504.0 / ((double)margin * (double)max_abs));
+    if (s < min_scale)
+        s = min_scale;
+    if (s > max_scale)
+        s = max_scale;
+    return s;
 }
 
 void orc_step(const uint16_t* const* grads, float* const* master,

@@ -75,6 +75,10 @@ typedef struct {
     uint64_t n_stale;    /* master moved but its FP16 copy did not            */
     float new_scale;     /* S for the next step                               */
     int32_t new_clean_run;
+    /* gradient statistics of pass 1 (the same read): */
+    uint16_t max_mag16;  /* largest |g16| bit pattern among finite gradients  */
+    float max_abs;       /* its unscaled value, fp32(max|g16|) * (1/S)        */
+    uint64_t exp_hist[32];/* count of gradients per binary16 exponent field  */
 } orc_result;
 
 /* Ablation mode of the test suite: update the FP16 weights directly, with no
@@ -99,6 +103,12 @@ uint64_t orc_update(int64_t count, const uint16_t* g16, float* w, float* v,
 /* Loss-scale state machine; returns the next S and updates *clean_run. */
 float orc_scaler_next(const orc_scaler_cfg* cfg, int32_t found_inf, float scale,
                       int32_t* clean_run);
+
+/* Direct choice of S from gradient statistics ("Choosing the Loss Scaling
+ * Factor", Method 2): S = 65504 / (margin * max|g|), in binary64, rounded to
+ * binary32 and clamped to [min_scale, max_scale]; max_abs == 0 gives 0 (no
+ * information: the caller keeps its S). */
+float orc_direct_scale(float max_abs, float margin, float min_scale, float max_scale);
 
 /* One whole step over a list of n tensors.  master/momentum/w16 are updated in
  * place unless the step overflows; r receives every output scalar. */

@@ -48,6 +48,11 @@ MUTANTS = [
     ("growth by backoff", "float s = scale * cfg->growth;", "float s = scale * cfg->backoff;"),
     ("stale test inverted", "h_new == orc_rne16(w_old)", "h_new != orc_rne16(w_old)"),
     ("fp16 copy from old weight", "uint16_t h_new = orc_rne16(wn);", "uint16_t h_new = orc_rne16(w_old);"),
+    ("histogram by fraction bits", "r->exp_hist[mag >> 10] += 1;", "r->exp_hist[mag & 31u] += 1;"),
+    ("maximum includes inf/NaN", "            if (mag > max_mag)   /* bit patterns of magnitudes order like values */\n                max_mag = mag;\n",
+     ""),
+    ("direct scale without margin", "(double)margin * (double)max_abs", "(double)max_abs"),
+    ("direct scale clamps swapped", "    if (s < min_scale)\n        s = min_scale;", "    if (s < min_scale)\n        s = max_scale;"),
 ]
 
 

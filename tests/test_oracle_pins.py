@@ -449,3 +449,45 @@ def test_p9_clip():
     expect = [f32(0.5) - (f32(-x) + f32(0.25)) for x in c.master]
     for x, y in zip(d.master, expect):
         assert np.array_equal(x, np.asarray(y, np.float32))
+
+
+# ---------------------------------------------------------------------------
+# Gradient statistics of pass 1 and the direct choice of S
+# ---------------------------------------------------------------------------
+
+def test_stats_histogram_and_max_against_numpy():
+    rng = np.random.default_rng(21)
+    g = rng.integers(0, 1 << 16, 50_000).astype(np.uint16)
+    g[:40] = [0, 0x8000, 0x0001, 0x7C00, 0xFC00, 0x7E00, 0x7BFF, 0xFBFF] * 5
+    parts = [g[:7], g[7:30_000], g[30_000:]]
+    r = oracle.check(parts, 2.0 ** 7)
+    mag = g & 0x7FFF
+    assert list(r.exp_hist) == np.bincount(mag >> 10, minlength=32).tolist()
+    finite = mag[mag < 0x7C00]
+    assert r.max_mag16 == finite.max() == 0x7BFF
+    expect = np.float32(np.array([finite.max()], np.uint16).view(np.float16)[0]) * np.float32(2.0 ** -7)
+    assert r.max_abs == expect
+    # the maximum ignores inf/NaN and is found in any tensor of the list
+    r2 = oracle.check([np.array([0x3C00, 0x7C00], np.uint16), np.array([0x4000], np.uint16)], 1.0)
+    assert (r2.max_mag16, r2.max_abs) == (0x4000, 2.0)
+
+
+def test_golden_direct_scale_formula():
+    F = facts()["direct_scale_formula"]
+    m = hx(F["max_abs_grad"])
+    assert oracle.direct_scale(m, margin=1.0) == hx(F["scale"])
+    assert oracle.direct_scale(m, margin=2.0) == hx(F["scale_with_margin"])
+    assert oracle.direct_scale(0.0) == 0.0                      # no information
+    assert oracle.direct_scale(2.0 ** -40, max_scale=2.0 ** 24) == 2.0 ** 24   # clamped
+    assert oracle.direct_scale(2.0 ** 40, min_scale=2.0 ** -24) == 2.0 ** -24
+
+
+@pytest.mark.parametrize("margin", [1.0, 2.0, 4.0])
+def test_direct_scale_puts_the_largest_gradient_at_65504_over_margin(margin):
+    rng = np.random.default_rng(int(margin))
+    g_true = (rng.standard_normal(4096) * 1e-2).astype(np.float32)
+    S = oracle.direct_scale(float(np.abs(g_true).max()), margin=margin)
+    scaled = oracle.rne16(g_true * np.float32(S))
+    assert np.all((scaled & 0x7FFF) < 0x7C00)                   # nothing overflows
+    top = float(oracle.widen16(scaled[np.argmax(np.abs(g_true))])[0])
+    assert abs(abs(top) - 65504.0 / margin) <= 32.0             # within half an ulp at 2^15
