@@ -23,15 +23,20 @@ _LIB = None
 NO_MASTER = 1  # ORC_NO_MASTER: ablation mode, FP16 weights updated directly
 
 
+SCALER_DYNAMIC, SCALER_DIRECT = 0, 1
+
+
 class ScalerCfg(ctypes.Structure):
     _fields_ = [("backoff", ctypes.c_float), ("growth", ctypes.c_float),
                 ("growth_interval", ctypes.c_int32), ("min_scale", ctypes.c_float),
-                ("max_scale", ctypes.c_float)]
+                ("max_scale", ctypes.c_float), ("mode", ctypes.c_int32),
+                ("direct_margin", ctypes.c_float)]
 
 
 def scaler_cfg(backoff=0.5, growth=2.0, growth_interval=0, min_scale=2.0 ** -24,
-               max_scale=2.0 ** 24):
-    return ScalerCfg(backoff, growth, growth_interval, min_scale, max_scale)
+               max_scale=2.0 ** 24, mode=SCALER_DYNAMIC, direct_margin=2.0):
+    return ScalerCfg(backoff, growth, growth_interval, min_scale, max_scale, mode,
+                     direct_margin)
 
 
 class _Result(ctypes.Structure):
@@ -68,7 +73,7 @@ def lib():
         L.orc_clip_coef.restype = None
         L.orc_update.argtypes = [i64, vp, vp, vp, vp, f32, i32, f32, f32, f32, f32, u32]
         L.orc_update.restype = ctypes.c_uint64
-        L.orc_scaler_next.argtypes = [ctypes.POINTER(ScalerCfg), i32, f32,
+        L.orc_scaler_next.argtypes = [ctypes.POINTER(ScalerCfg), i32, f32, f32,
                                       ctypes.POINTER(ctypes.c_int32)]
         L.orc_scaler_next.restype = f32
         L.orc_step.argtypes = [vp, vp, vp, vp, vp, i32, f32, f32, f32, f32, f32,
@@ -166,9 +171,9 @@ def direct_scale(max_abs, margin=2.0, min_scale=2.0 ** -24, max_scale=2.0 ** 24)
     return lib().orc_direct_scale(max_abs, margin, min_scale, max_scale)
 
 
-def scaler_next(cfg, found_inf, scale, clean_run):
+def scaler_next(cfg, found_inf, scale, clean_run, max_abs=0.0):
     c = ctypes.c_int32(clean_run)
-    s = lib().orc_scaler_next(ctypes.byref(cfg), int(found_inf), scale, ctypes.byref(c))
+    s = lib().orc_scaler_next(ctypes.byref(cfg), int(found_inf), max_abs, scale, ctypes.byref(c))
     return s, c.value
 
 

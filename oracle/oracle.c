@@ -213,8 +213,8 @@ uint64_t orc_update(int64_t count, const uint16_t* g16, float* w, float* v,
     return stale;
 }
 
-float orc_scaler_next(const orc_scaler_cfg* cfg, int32_t found_inf, float scale,
-                      int32_t* clean_run)
+float orc_scaler_next(const orc_scaler_cfg* cfg, int32_t found_inf, float max_abs,
+                      float scale, int32_t* clean_run)
 {
     /* Method 3 of "Choosing the Loss Scaling Factor" and the tutorial's
      * dynamic rule: on overflow skip and multiply S by beta; after N
@@ -226,6 +226,12 @@ float orc_scaler_next(const orc_scaler_cfg* cfg, int32_t found_inf, float scale,
         return s < cfg->min_scale ? cfg->min_scale : s;
     }
     *clean_run += 1;
+    if (cfg->mode == ORC_SCALER_DIRECT) {
+        /* Method 2 with this step's own statistics standing in for those of
+         * an FP32 run; no information (all gradients zero) keeps S. */
+        float s = orc_direct_scale(max_abs, cfg->direct_margin, cfg->min_scale, cfg->max_scale);
+        return s > 0.0f ? s : scale;
+    }
     if (cfg->growth_interval > 0 && *clean_run >= cfg->growth_interval) {
         float s = scale * cfg->growth;
         *clean_run = 0;
@@ -269,6 +275,6 @@ void orc_step(const uint16_t* const* grads, float* const* master,
                                      r->clip_coef, lr, momentum_coef,
                                      weight_decay, flags);
     }
-    r->new_scale = orc_scaler_next(cfg, r->found_inf, scale, clean_run);
+    r->new_scale = orc_scaler_next(cfg, r->found_inf, r->max_abs, scale, clean_run);
     r->new_clean_run = *clean_run;
 }

@@ -61,7 +61,13 @@ typedef struct {
     int32_t growth_interval; /* N; 0 = never grow (constant S)               */
     float min_scale;         /* floor on S after a backoff                    */
     float max_scale;         /* ceiling on S after a growth                   */
+    int32_t mode;            /* ORC_SCALER_DYNAMIC or ORC_SCALER_DIRECT       */
+    float direct_margin;     /* direct mode: S = 65504 / (margin * max|g|)    */
 } orc_scaler_cfg;
+
+#define ORC_SCALER_DYNAMIC 0 /* Method 3: backoff on overflow, growth after N */
+#define ORC_SCALER_DIRECT 1  /* Method 2 from each step's own max|g|; backoff
+                                on overflow                                   */
 
 typedef struct {
     int32_t found_inf;   /* any +-inf/NaN anywhere in the list                */
@@ -100,9 +106,10 @@ uint64_t orc_update(int64_t count, const uint16_t* g16, float* w, float* v,
                     uint16_t* w16, float inv_scale, int32_t clipped, float coef,
                     float lr, float momentum, float weight_decay, uint32_t flags);
 
-/* Loss-scale state machine; returns the next S and updates *clean_run. */
-float orc_scaler_next(const orc_scaler_cfg* cfg, int32_t found_inf, float scale,
-                      int32_t* clean_run);
+/* Loss-scale state machine; returns the next S and updates *clean_run.
+ * max_abs (the step's largest unscaled finite |g|) is used by direct mode. */
+float orc_scaler_next(const orc_scaler_cfg* cfg, int32_t found_inf, float max_abs,
+                      float scale, int32_t* clean_run);
 
 /* Direct choice of S from gradient statistics ("Choosing the Loss Scaling
  * Factor", Method 2): S = 65504 / (margin * max|g|), in binary64, rounded to

@@ -53,6 +53,8 @@ MUTANTS = [
      ""),
     ("direct scale without margin", "(double)margin * (double)max_abs", "(double)max_abs"),
     ("direct scale clamps swapped", "    if (s < min_scale)\n        s = min_scale;", "    if (s < min_scale)\n        s = max_scale;"),
+    ("direct mode ignored", "    if (cfg->mode == ORC_SCALER_DIRECT) {", "    if (0) {"),
+    ("direct mode zero max gives zero", "        return s > 0.0f ? s : scale;", "        return s;"),
 ]
 
 

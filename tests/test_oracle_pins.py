@@ -491,3 +491,21 @@ def test_direct_scale_puts_the_largest_gradient_at_65504_over_margin(margin):
     assert np.all((scaled & 0x7FFF) < 0x7C00)                   # nothing overflows
     top = float(oracle.widen16(scaled[np.argmax(np.abs(g_true))])[0])
     assert abs(abs(top) - 65504.0 / margin) <= 32.0             # within half an ulp at 2^15
+
+
+def test_direct_scaler_mode_through_the_step():
+    """Direct mode: after a clean step S = 65504 / (margin * max|g_true|) of
+    that step; an overflow backs off; all-zero gradients keep S."""
+    cfg = oracle.scaler_cfg(mode=oracle.SCALER_DIRECT, direct_margin=2.0)
+    st = one_tensor_state([0.5, -0.25, 1.0])
+    S = 2.0 ** 10
+    g_true = np.array([2.0 ** -9, -(2.0 ** -6), 3 * 2.0 ** -12], np.float32)
+    r = oracle.step(st, [oracle.rne16(g_true * np.float32(S))], S, 0.01, 0.9, 0.0, cfg=cfg)
+    assert r["max_abs"] == 2.0 ** -6
+    assert r["new_scale"] == np.float32(65504.0 / (2.0 * 2.0 ** -6))
+    S2 = r["new_scale"]
+    bad = np.array([0x7C00, 0, 0], np.uint16)
+    r = oracle.step(st, [bad], S2, 0.01, 0.9, 0.0, cfg=cfg)
+    assert r["found_inf"] == 1 and r["new_scale"] == S2 * 0.5
+    r = oracle.step(st, [np.zeros(3, np.uint16)], 64.0, 0.01, 0.9, 0.0, cfg=cfg)
+    assert r["max_abs"] == 0.0 and r["new_scale"] == 64.0
