@@ -21,6 +21,8 @@ from . import build as _build
 _LIB = None
 
 NO_MASTER = 1  # ORC_NO_MASTER: ablation mode, FP16 weights updated directly
+NESTEROV = 2   # ORC_NESTEROV: Nesterov momentum
+ADAGRAD = 4    # ORC_ADAGRAD: Adagrad (the momentum array holds sum of d^2)
 
 
 SCALER_DYNAMIC, SCALER_DIRECT = 0, 1
@@ -71,12 +73,12 @@ def lib():
         L.orc_check.restype = None
         L.orc_clip_coef.argtypes = [ctypes.POINTER(_Result), f32]
         L.orc_clip_coef.restype = None
-        L.orc_update.argtypes = [i64, vp, vp, vp, vp, f32, i32, f32, f32, f32, f32, u32]
+        L.orc_update.argtypes = [i64, vp, vp, vp, vp, f32, i32, f32, f32, f32, f32, f32, u32]
         L.orc_update.restype = ctypes.c_uint64
         L.orc_scaler_next.argtypes = [ctypes.POINTER(ScalerCfg), i32, f32, f32,
                                       ctypes.POINTER(ctypes.c_int32)]
         L.orc_scaler_next.restype = f32
-        L.orc_step.argtypes = [vp, vp, vp, vp, vp, i32, f32, f32, f32, f32, f32,
+        L.orc_step.argtypes = [vp, vp, vp, vp, vp, i32, f32, f32, f32, f32, f32, f32,
                                ctypes.POINTER(ScalerCfg), ctypes.POINTER(ctypes.c_int32),
                                u32, ctypes.POINTER(_Result)]
         L.orc_step.restype = None
@@ -156,14 +158,15 @@ def clip_coef(r, clip):
     return r
 
 
-def update(g16, w, v, w16, scale, clipped, coef, lr, momentum, weight_decay, flags=0):
+def update(g16, w, v, w16, scale, clipped, coef, lr, momentum, weight_decay, flags=0,
+           eps=1e-10):
     """Pass 2 on one set of elements (arrays are updated in place)."""
     g16 = _c(g16, np.uint16)
     for a, dt in ((w, np.float32), (v, np.float32), (w16, np.uint16)):
         assert a.flags.c_contiguous and a.dtype == dt
     inv = np.float32(1.0) / np.float32(scale)
     return lib().orc_update(g16.size, _ptr(g16), _ptr(w), _ptr(v), _ptr(w16), inv,
-                            int(clipped), coef, lr, momentum, weight_decay, flags)
+                            int(clipped), coef, lr, momentum, weight_decay, eps, flags)
 
 
 def direct_scale(max_abs, margin=2.0, min_scale=2.0 ** -24, max_scale=2.0 ** 24):
@@ -177,7 +180,8 @@ def scaler_next(cfg, found_inf, scale, clean_run, max_abs=0.0):
     return s, c.value
 
 
-def step(state, grads, scale, lr, momentum, weight_decay, clip=0.0, cfg=None, flags=0):
+def step(state, grads, scale, lr, momentum, weight_decay, clip=0.0, cfg=None, flags=0,
+         eps=1e-10):
     """One whole step; ``state`` is updated in place.  Returns the result dict."""
     cfg = cfg if cfg is not None else scaler_cfg()
     grads = [_c(g, np.uint16) for g in grads]
@@ -191,7 +195,7 @@ def step(state, grads, scale, lr, momentum, weight_decay, clip=0.0, cfg=None, fl
     master = _ptr_array(state.master) if not (flags & NO_MASTER) else None
     lib().orc_step(_ptr_array(grads), master, _ptr_array(state.momentum),
                    _ptr_array(state.w16), _ptr(sizes), n, scale, lr, momentum,
-                   weight_decay, clip, ctypes.byref(cfg), ctypes.byref(clean), flags,
+                   weight_decay, clip, eps, ctypes.byref(cfg), ctypes.byref(clean), flags,
                    ctypes.byref(r))
     state.clean_run = clean.value
     state.scale_history.append(r.new_scale)

@@ -183,7 +183,8 @@ void orc_clip_coef(orc_result* r, float clip)
 
 uint64_t orc_update(int64_t count, const uint16_t* g16, float* w, float* v,
                     uint16_t* w16, float inv_scale, int32_t clipped, float coef,
-                    float lr, float momentum, float weight_decay, uint32_t flags)
+                    float lr, float momentum, float weight_decay, float eps,
+                    uint32_t flags)
 {
     uint64_t stale = 0;
     for (int64_t j = 0; j < count; ++j) {
@@ -196,9 +197,25 @@ uint64_t orc_update(int64_t count, const uint16_t* g16, float* w, float* v,
 
         float t = weight_decay * w_old;                /* g_eff = g + lambda*w */
         float d = g + t;
-        float u = momentum * v[j];                     /* v_t = mu*v_{t-1} + g */
-        float vn = u + d;
-        float s = lr * vn;                             /* w = w - eta*v_t      */
+        float vn, step;
+        if (flags & ORC_ADAGRAD) {
+            /* Adagrad: the state is the running sum of squared gradients,
+             * h = h + d^2, and the step is d / (sqrt(h) + eps). */
+            float sq = d * d;
+            vn = v[j] + sq;
+            float den = sqrtf(vn) + eps;
+            step = d / den;
+        } else {
+            float u = momentum * v[j];                 /* v_t = mu*v_{t-1} + g */
+            vn = u + d;
+            step = vn;
+            if (flags & ORC_NESTEROV) {
+                /* Nesterov momentum: step along d + mu * v_t */
+                float m2 = momentum * vn;
+                step = d + m2;
+            }
+        }
+        float s = lr * step;                           /* w = w - eta*v_t      */
         float wn = w_old - s;
 
         v[j] = vn;
@@ -257,7 +274,7 @@ float orc_direct_scale(float max_abs, float margin, float min_scale, float max_s
 void orc_step(const uint16_t* const* grads, float* const* master,
               float* const* momentum, uint16_t* const* w16, const int64_t* sizes,
               int32_t n, float scale, float lr, float momentum_coef,
-              float weight_decay, float clip, const orc_scaler_cfg* cfg,
+              float weight_decay, float clip, float eps, const orc_scaler_cfg* cfg,
               int32_t* clean_run, uint32_t flags, orc_result* r)
 {
     float inv_scale = 1.0f / scale;
@@ -273,7 +290,7 @@ void orc_step(const uint16_t* const* grads, float* const* master,
             r->n_stale += orc_update(sizes[i], grads[i], master ? master[i] : NULL,
                                      momentum[i], w16[i], inv_scale, r->clipped,
                                      r->clip_coef, lr, momentum_coef,
-                                     weight_decay, flags);
+                                     weight_decay, eps, flags);
     }
     r->new_scale = orc_scaler_next(cfg, r->found_inf, r->max_abs, scale, clean_run);
     r->new_clean_run = *clean_run;

@@ -91,6 +91,17 @@ typedef struct {
  * FP32 master copy (the configuration the pages compare against). */
 #define ORC_NO_MASTER 1u
 
+/* Optimizer of the update (default: SGD with momentum, Step 7 of "The
+ * Integrated Training Procedure (Figure 1)").  The pages' speech models used
+ * Nesterov SGD and the bigLSTM Adagrad (section 5 of the analysis, model
+ * descriptions); neither formula is printed there, so these are the standard
+ * forms, each operation rounded to binary32:
+ *   Nesterov: v = mu*v + d;  w = w - eta*(d + mu*v)
+ *   Adagrad:  h = h + d*d;   w = w - eta*d/(sqrt(h) + eps)   (h in the
+ *             momentum array, h0 = 0) */
+#define ORC_NESTEROV 2u
+#define ORC_ADAGRAD 4u
+
 /* Pass 1 (Steps 5-6): overflow check, range counts and the sum of squares of
  * fp32(g16) * inv_scale over every tensor of the list, in list order. */
 void orc_check(const uint16_t* const* grads, const int64_t* sizes, int32_t n,
@@ -104,7 +115,8 @@ void orc_clip_coef(orc_result* r, float clip);
  * of "stale" elements (master moved, FP16 copy did not). */
 uint64_t orc_update(int64_t count, const uint16_t* g16, float* w, float* v,
                     uint16_t* w16, float inv_scale, int32_t clipped, float coef,
-                    float lr, float momentum, float weight_decay, uint32_t flags);
+                    float lr, float momentum, float weight_decay, float eps,
+                    uint32_t flags);
 
 /* Loss-scale state machine; returns the next S and updates *clean_run.
  * max_abs (the step's largest unscaled finite |g|) is used by direct mode. */
@@ -122,7 +134,7 @@ float orc_direct_scale(float max_abs, float margin, float min_scale, float max_s
 void orc_step(const uint16_t* const* grads, float* const* master,
               float* const* momentum, uint16_t* const* w16, const int64_t* sizes,
               int32_t n, float scale, float lr, float momentum_coef,
-              float weight_decay, float clip, const orc_scaler_cfg* cfg,
+              float weight_decay, float clip, float eps, const orc_scaler_cfg* cfg,
               int32_t* clean_run, uint32_t flags, orc_result* r);
 
 #ifdef __cplusplus

@@ -22,10 +22,10 @@ MUTANTS = [
     ("weight decay sign", "float d = g + t;", "float d = g - t;"),
     ("weight decay dropped", "float d = g + t;", "float d = g;"),
     ("weight decay on momentum", "float t = weight_decay * w_old;", "float t = weight_decay * v[j];"),
-    ("momentum term dropped", "float vn = u + d;", "float vn = d;"),
+    ("momentum term dropped", "vn = u + d;", "vn = d;"),
     ("momentum on gradient", "float u = momentum * v[j];", "float u = momentum * d;"),
     ("update sign", "float wn = w_old - s;", "float wn = w_old + s;"),
-    ("update uses d not v", "float s = lr * vn;", "float s = lr * d;"),
+    ("update uses d not v", "step = vn;", "step = d;"),
     ("unscale dropped", "return orc_widen16(g16) * inv_scale;", "return orc_widen16(g16);"),
     ("clip inverted", "g = g * coef;", "g = g / coef;"),
     ("clip coefficient inverted", "r->clip_coef = (float)((double)clip / r->norm);",
@@ -55,6 +55,12 @@ MUTANTS = [
     ("direct scale clamps swapped", "    if (s < min_scale)\n        s = min_scale;", "    if (s < min_scale)\n        s = max_scale;"),
     ("direct mode ignored", "    if (cfg->mode == ORC_SCALER_DIRECT) {", "    if (0) {"),
     ("direct mode zero max gives zero", "        return s > 0.0f ? s : scale;", "        return s;"),
+    ("nesterov look-ahead dropped", "                step = d + m2;", "                step = vn;"),
+    ("nesterov look-ahead on old v", "float m2 = momentum * vn;", "float m2 = momentum * v[j];"),
+    ("adagrad without square", "float sq = d * d;", "float sq = d;"),
+    ("adagrad without root", "float den = sqrtf(vn) + eps;", "float den = vn + eps;"),
+    ("adagrad eps inside root", "float den = sqrtf(vn) + eps;", "float den = sqrtf(vn + eps);"),
+    ("adagrad accumulates before decay", "            float sq = d * d;", "            float sq = g * g;"),
 ]
 
 

@@ -509,3 +509,95 @@ def test_direct_scaler_mode_through_the_step():
     assert r["found_inf"] == 1 and r["new_scale"] == S2 * 0.5
     r = oracle.step(st, [np.zeros(3, np.uint16)], 64.0, 0.01, 0.9, 0.0, cfg=cfg)
     assert r["max_abs"] == 0.0 and r["new_scale"] == 64.0
+
+
+# ---------------------------------------------------------------------------
+# Nesterov momentum and Adagrad (the pages' speech models and bigLSTM)
+# ---------------------------------------------------------------------------
+
+def brute_force_update(w, v, g16, S, lr, mom, wd, opt, eps=1e-10):
+    """Python restatement of one update, each binary32 op correctly rounded
+    via binary64 (sqrt too: binary64 has more than 2*24+2 bits)."""
+    S, lr, mom, wd, eps = (float(f32(x)) for x in (S, lr, mom, wd, eps))
+    inv = float(f32(1.0 / S))
+    W, V = [], []
+    for h, wi, vi in zip(g16, w.tolist(), v.tolist()):
+        g = float(f32(_bf_widen(h) * inv))
+        d = float(f32(g + float(f32(wd * wi))))
+        if opt == "adagrad":
+            vn = float(f32(vi + float(f32(d * d))))
+            den = float(f32(float(f32(math.sqrt(vn))) + eps))
+            step = float(f32(d / den))
+        else:
+            vn = float(f32(float(f32(mom * vi)) + d))
+            step = vn if opt == "momentum" else float(f32(d + float(f32(mom * vn))))
+        W.append(float(f32(wi - float(f32(lr * step)))))
+        V.append(vn)
+    return np.array(W, np.float32), np.array(V, np.float32)
+
+
+@pytest.mark.parametrize("opt,flag", [("nesterov", oracle.NESTEROV), ("adagrad", oracle.ADAGRAD),
+                                      ("momentum", 0)])
+def test_optimizers_brute_force(opt, flag):
+    rng = np.random.default_rng(77)
+    n = 64
+    w = rng.normal(0, 0.05, n).astype(np.float32)
+    st = oracle.State.from_master([w])
+    bw, bv = w.copy(), np.zeros(n, np.float32)
+    for step in range(5):
+        g16 = ((rng.integers(0, 2, n) << 15) | (rng.integers(1, 29, n) << 10) |
+               rng.integers(0, 1024, n)).astype(np.uint16)
+        r = oracle.step(st, [g16], 2.0 ** 6, 0.01, 0.9, 1e-4, flags=flag)
+        assert r["found_inf"] == 0
+        bw, bv = brute_force_update(bw, bv, g16, 2.0 ** 6, 0.01, 0.9, 1e-4, opt)
+        assert st.master[0].tobytes() == bw.tobytes(), (opt, step)
+        assert st.momentum[0].tobytes() == bv.tobytes(), (opt, step)
+        assert st.w16[0].tobytes() == oracle.rne16(bw).tobytes()
+
+
+def test_nesterov_exact_recurrence():
+    """v_t = mu v + d;  w_t = w - eta (d + mu v_t) in exact rationals while
+    every intermediate is a binary32 number."""
+    mu, lr, S = Fraction(1, 2), Fraction(1, 4), Fraction(2)
+    g16 = np.array([0x3E00, 0xB800], np.uint16)                 # 1.5, -0.5
+    g = [Fraction(_bf_widen(h)) / S for h in g16]
+    w, v = [Fraction(1), Fraction(-3, 4)], [Fraction(0)] * 2
+    st = oracle.State.from_master([np.array([float(x) for x in w], np.float32)])
+    exact = 0
+    for _ in range(10):
+        nv = [mu * v[i] + g[i] for i in range(2)]
+        stepv = [g[i] + mu * nv[i] for i in range(2)]
+        nw = [w[i] - lr * stepv[i] for i in range(2)]
+        if not all(_exact_f32(x) for x in nv + stepv + nw + [lr * s for s in stepv]):
+            break
+        oracle.step(st, [g16], float(S), float(lr), float(mu), 0.0, flags=oracle.NESTEROV)
+        w, v = nw, nv
+        assert [Fraction(float(x)) for x in st.master[0]] == w
+        exact += 1
+    assert exact >= 4
+
+
+def test_adagrad_first_step_is_lr_times_sign():
+    """With h0 = 0 and eps = 0 the first Adagrad step is exactly eta * sign(d)
+    whatever the gradient's size; afterwards h holds the sum of squares."""
+    g_true = np.array([3e-5, -7.0, 2.0 ** -20, -0.25], np.float32)
+    g16 = oracle.rne16(g_true * f32(1024))
+    st = oracle.State.from_master([np.full(4, 0.5, np.float32)])
+    oracle.step(st, [g16], 1024.0, 0.125, 0.0, 0.0, flags=oracle.ADAGRAD, eps=0.0)
+    assert st.master[0].tolist() == [0.5 - 0.125, 0.5 + 0.125, 0.5 - 0.125, 0.5 + 0.125]
+    g = oracle.widen16(g16) * f32(2.0 ** -10)
+    assert np.array_equal(st.momentum[0], g * g)
+    oracle.step(st, [g16], 1024.0, 0.125, 0.0, 0.0, flags=oracle.ADAGRAD, eps=0.0)
+    assert np.array_equal(st.momentum[0], g * g + g * g)
+
+
+def test_adagrad_closed_form_constant_gradient():
+    # constant g: h_t = t g^2, w_t = w0 - eta sum_k g / (sqrt(k) |g| + eps)
+    g16 = np.array([0x2C00], np.uint16)                          # 2^-4
+    st = oracle.State.from_master([np.array([1.0], np.float32)])
+    w, eps, lr = 1.0, float(f32(1e-10)), float(f32(0.01))
+    for t in range(1, 21):
+        oracle.step(st, [g16], 1.0, 0.01, 0.0, 0.0, flags=oracle.ADAGRAD)
+        w -= lr * 2.0 ** -4 / (math.sqrt(t) * 2.0 ** -4 + eps)
+        assert abs(float(st.master[0][0]) - w) <= 4 * t * float(np.spacing(f32(w)))
+    assert float(st.momentum[0][0]) == 20 * 2.0 ** -8
