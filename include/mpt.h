@@ -64,6 +64,33 @@ extern "C" {
                                      against the tensor sizes and arenas     */
 #define MPT_FLAG_COUNT_STALE 0x2u /* count elements whose master moved but
                                      whose FP16 copy did not                 */
+#define MPT_FLAG_GRAD_STATS 0x4u  /* the check pass also finds the largest
+                                     |g16| and counts the gradients per
+                                     binary16 exponent field (see
+                                     mpt_grad_histogram); implied by
+                                     MPT_SCALER_DIRECT                      */
+
+/* Loss-scale modes ("Choosing the Loss Scaling Factor").  Both skip the
+ * update and multiply S by backoff on overflow.
+ *   DYNAMIC (Method 3): after growth_interval consecutive clean steps,
+ *     multiply S by growth.
+ *   DIRECT (Method 2): after every clean step set S = 65504 / (margin *
+ *     max|g|), max|g| being that step's largest unscaled finite gradient
+ *     (binary64, rounded to binary32, clamped to [min_scale, max_scale]);
+ *     a step whose gradients are all zero keeps S. */
+#define MPT_SCALER_DYNAMIC 0
+#define MPT_SCALER_DIRECT 1
+
+/* Update rule of the FP32 master (every operation rounded to binary32; d is
+ * the unscaled, clipped gradient plus weight decay, d = g + lambda*w):
+ *   MOMENTUM (default; Step 7): v = mu*v + d;  w = w - eta*v
+ *   NESTEROV (the pages' speech models): v = mu*v + d;  w = w - eta*(d + mu*v)
+ *   ADAGRAD (the pages' bigLSTM): v = v + d*d;  w = w - eta*d/(sqrt(v) + eps)
+ *     -- the momentum arena holds the running sum of squares (zero at
+ *     creation) and the momentum argument of the step is ignored. */
+#define MPT_OPT_MOMENTUM 0
+#define MPT_OPT_NESTEROV 1
+#define MPT_OPT_ADAGRAD 2
 
 typedef struct {
     float backoff;            /* beta: S multiplier on overflow (default 0.5)      */
@@ -74,6 +101,11 @@ typedef struct {
     uint32_t flags;           /* MPT_FLAG_* (default 0)                            */
     int32_t chunk_elems;      /* elements per work bin: a multiple of 2048 in
                                  [2048, 2^20]; 0 = default (32768)                 */
+    int32_t scaler_mode;      /* MPT_SCALER_DYNAMIC (default) or _DIRECT           */
+    float direct_margin;      /* direct mode: margin > 0 (default 2: one bit of
+                                 headroom, as the pages suggest)                   */
+    int32_t optimizer;        /* MPT_OPT_MOMENTUM (default), _NESTEROV, _ADAGRAD   */
+    float eps;                /* Adagrad denominator term (default 1e-10)          */
 } mpt_config;
 
 /* ---- results ------------------------------------------------------------ */
@@ -86,7 +118,8 @@ typedef struct {
     double grad_norm;      /* global L2 norm of the unscaled, unclipped
                               gradients; +inf when found_inf                    */
     float clip_coef;       /* clip / grad_norm when clipped, else 1             */
-    int32_t reserved;
+    float max_abs_grad;    /* MPT_FLAG_GRAD_STATS / direct mode, else 0: the
+                              largest unscaled finite |g|, fp32(max|g16|)*(1/S) */
     uint64_t n_zero;       /* FP16 gradients equal to +-0                       */
     uint64_t n_subnormal;  /* FP16 gradients with 0 < |g16| < 2^-14             */
     uint64_t n_nonfinite;  /* FP16 gradients that are +-inf or NaN              */
@@ -157,7 +190,7 @@ int mpt_refresh_half(mpt_handle* h, void* cuda_stream);
  * by `scale` (any 2-byte alignment; contents are only read).  lr, momentum
  * and weight_decay are eta, mu and lambda; clip <= 0 disables clipping.
  * Work is queued on cuda_stream and the call waits for it (it reads the
- * 112-byte control block back).  The scale state advances from `scale`:
+ * 128-byte control block back).  The scale state advances from `scale`:
  * out->new_scale is the S for the next step.  On overflow the arenas are
  * untouched.  Errors: MPT_ERR_INVALID_ARG, MPT_ERR_CUDA,
  * MPT_ERR_DEVICE_CHECK (checked mode; the bins that passed their check were
@@ -186,6 +219,61 @@ int mpt_wait(mpt_handle* h, void* cuda_stream, mpt_step_result* out);
  * mpt_step_async uses (inside the workspace): a training loop multiplies its
  * loss by it on the device.  Errors: MPT_ERR_INVALID_ARG. */
 int mpt_device_scale(const mpt_handle* h, float** d_scale);
+
+/* ---- sharded step (optimizer state split across the ranks of a data-
+ * parallel group) ---------------------------------------------------------
+ *
+ * The flat parameter list (all tensors concatenated, P elements) is cut into
+ * `world` equal contiguous shards of mpt_shard_len(P, world) elements (the
+ * last one padded with elements whose gradient is always zero).  Rank r
+ * creates an ordinary handle over ONE tensor of shard_len elements: it owns
+ * the FP32 master, FP32 momentum and FP16 copy of flat elements
+ * [r*shard_len, (r+1)*shard_len).  Per step, with the loss scale on the
+ * device (as mpt_step_async):
+ *   1. the caller reduce-scatters the FP16 gradients so that each rank holds
+ *      the summed gradients of its shard (an FP16 sum can itself overflow;
+ *      step 2 catches it like any other inf);
+ *   2. mpt_step_partial queues the check pass over the shard and returns the
+ *      device address of its 32-byte record (MPT_PARTIAL_BYTES: binary64 sum
+ *      of squares, non-finite count, largest finite |g16|, error bits);
+ *   3. the caller all-gathers the records of all ranks, in rank order, into
+ *      one device array (16-byte aligned);
+ *   4. mpt_step_finish adds the records in rank order (so every rank gets
+ *      bit-identical totals and the same next S), finishes the step and
+ *      queues the update of the shard;
+ *   5. the caller all-gathers the FP16 copies of the shards.
+ * Only 32 bytes per rank cross between the two kernels of a step.  The
+ * halves are not timed by mpt_set_timing; mpt_wait returns the last result:
+ * found_inf, n_nonfinite, grad_norm, the clip coefficient and the scale are
+ * those of the whole list (equal on every rank), n_zero, n_subnormal and the
+ * histogram those of this rank's shard. */
+#define MPT_PARTIAL_BYTES 32
+
+/* shard_len = ceil(total / world) rounded up to a multiple of 16.
+ * Errors: MPT_ERR_INVALID_ARG. */
+int mpt_shard_len(int64_t total, int32_t world, int64_t* shard_len);
+
+/* Phase 2: queue the check pass over the handle's gradients (a host array of
+ * its tensors' device pointers, as for mpt_step) with S from the device
+ * state; *d_partial receives the device address of this rank's record
+ * (valid until the next call on the handle).  Errors: MPT_ERR_INVALID_ARG,
+ * MPT_ERR_CUDA, MPT_ERR_BROKEN. */
+int mpt_step_partial(mpt_handle* h, const void* const* d_grads_half, void* cuda_stream,
+                     void** d_partial);
+
+/* Phase 4: d_partials = device array of `world` records in rank order;
+ * finishes the step (norm, clip coefficient, loss-scale state) and queues the
+ * update over the gradients of the preceding mpt_step_partial.
+ * Errors: MPT_ERR_INVALID_ARG (no check pass queued, misaligned records),
+ * MPT_ERR_CUDA, MPT_ERR_BROKEN. */
+int mpt_step_finish(mpt_handle* h, const void* d_partials, int32_t world, float lr,
+                    float momentum, float weight_decay, float clip, void* cuda_stream);
+
+/* Statistics mode: counts[e] = number of gradients of the last step whose
+ * binary16 exponent field is e (e = 0: zeros and subnormals; e = 31: inf and
+ * NaN; otherwise |g16| in [2^(e-15), 2^(e-14))), as of the last waiting
+ * call; all zero without statistics.  Errors: MPT_ERR_INVALID_ARG. */
+int mpt_grad_histogram(const mpt_handle* h, uint64_t counts[32]);
 
 /* Counters and the last result, as of the last waiting call.
  * Errors: MPT_ERR_INVALID_ARG. */

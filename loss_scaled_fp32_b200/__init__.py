@@ -19,10 +19,18 @@ import os
 from . import build as _build
 
 __all__ = ["MPT", "Config", "MptError", "lib", "grad_pointers", "check_flat_noalloc",
-           "MPT_FLAG_CHECKED", "MPT_FLAG_COUNT_STALE"]
+           "MPT_FLAG_CHECKED", "MPT_FLAG_COUNT_STALE", "MPT_FLAG_GRAD_STATS",
+           "MPT_SCALER_DYNAMIC", "MPT_SCALER_DIRECT", "MPT_OPT_MOMENTUM", "MPT_OPT_NESTEROV",
+           "MPT_OPT_ADAGRAD"]
 
 MPT_FLAG_CHECKED = 0x1
 MPT_FLAG_COUNT_STALE = 0x2
+MPT_FLAG_GRAD_STATS = 0x4
+MPT_SCALER_DYNAMIC = 0
+MPT_SCALER_DIRECT = 1
+MPT_OPT_MOMENTUM = 0
+MPT_OPT_NESTEROV = 1
+MPT_OPT_ADAGRAD = 2
 
 MPT_OK = 0
 MPT_ERR_INVALID_ARG = -1
@@ -32,6 +40,7 @@ MPT_ERR_DEVICE_CHECK = -4
 MPT_ERR_BROKEN = -5
 MPT_ERR_TOO_LARGE = -6
 MPT_NOALLOC_MAX_ELEMS = 1 << 30
+MPT_PARTIAL_BYTES = 32
 
 
 class MptError(RuntimeError):
@@ -44,7 +53,9 @@ class Config(ctypes.Structure):
     _fields_ = [("backoff", ctypes.c_float), ("growth", ctypes.c_float),
                 ("growth_interval", ctypes.c_int32), ("min_scale", ctypes.c_float),
                 ("max_scale", ctypes.c_float), ("flags", ctypes.c_uint32),
-                ("chunk_elems", ctypes.c_int32)]
+                ("chunk_elems", ctypes.c_int32), ("scaler_mode", ctypes.c_int32),
+                ("direct_margin", ctypes.c_float), ("optimizer", ctypes.c_int32),
+                ("eps", ctypes.c_float)]
 
     def __init__(self, **kw):
         super().__init__()
@@ -59,12 +70,12 @@ class StepResult(ctypes.Structure):
     _fields_ = [("found_inf", ctypes.c_int32), ("clipped", ctypes.c_int32),
                 ("new_scale", ctypes.c_float), ("clean_run", ctypes.c_int32),
                 ("grad_norm", ctypes.c_double), ("clip_coef", ctypes.c_float),
-                ("reserved", ctypes.c_int32), ("n_zero", ctypes.c_uint64),
+                ("max_abs_grad", ctypes.c_float), ("n_zero", ctypes.c_uint64),
                 ("n_subnormal", ctypes.c_uint64), ("n_nonfinite", ctypes.c_uint64),
                 ("n_fp16_stale", ctypes.c_uint64)]
 
     def as_dict(self):
-        return {k: getattr(self, k) for k, _ in self._fields_ if k != "reserved"}
+        return {k: getattr(self, k) for k, _ in self._fields_}
 
 
 class CheckResult(ctypes.Structure):
@@ -118,6 +129,10 @@ def lib():
             "mpt_step_async": [vp, vp, f32, f32, f32, f32, vp],
             "mpt_wait": [vp, vp, ctypes.POINTER(StepResult)],
             "mpt_device_scale": [vp, ctypes.POINTER(vp)],
+            "mpt_grad_histogram": [vp, ctypes.POINTER(ctypes.c_uint64 * 32)],
+            "mpt_shard_len": [ctypes.c_int64, i32, ctypes.POINTER(ctypes.c_int64)],
+            "mpt_step_partial": [vp, vp, vp, ctypes.POINTER(vp)],
+            "mpt_step_finish": [vp, vp, i32, f32, f32, f32, f32, vp],
         }
         for name, args in sig.items():
             fn = getattr(L, name)
@@ -151,6 +166,13 @@ def check_flat_noalloc(grads, scale, clip, out, stream=None):
                                         scale, clip, ctypes.c_void_p(out.data_ptr()),
                                         _stream_ptr(stream, grads.device)),
            "mpt_check_flat_noalloc")
+
+
+def shard_len(total, world):
+    """Elements per rank of the sharded step (``mpt_shard_len``)."""
+    n = ctypes.c_int64()
+    _check(lib().mpt_shard_len(int(total), int(world), ctypes.byref(n)), "mpt_shard_len")
+    return n.value
 
 
 def _stream_ptr(stream, device):
@@ -253,6 +275,29 @@ class MPT:
         off = p.value - self.workspace.data_ptr()
         import torch
         return self.workspace[off:off + 4].view(torch.float32)
+
+    def step_partial(self, grads, stream=None):
+        """Sharded step, phase 2: queue the check pass; returns a 32-byte
+        uint8 CUDA tensor aliasing this rank's record."""
+        import torch
+        p = ctypes.c_void_p()
+        _check(lib().mpt_step_partial(self._h, self._ptrs(grads), _stream_ptr(stream, self.device),
+                                      ctypes.byref(p)), "mpt_step_partial")
+        off = p.value - self.workspace.data_ptr()
+        return self.workspace[off:off + MPT_PARTIAL_BYTES]
+
+    def step_finish(self, partials, world, lr, momentum, weight_decay, clip=0.0, stream=None):
+        """Sharded step, phase 4: ``partials`` is a CUDA tensor holding the
+        ``world`` records in rank order."""
+        _check(lib().mpt_step_finish(self._h, ctypes.c_void_p(partials.data_ptr()), world, lr,
+                                     momentum, weight_decay, clip,
+                                     _stream_ptr(stream, self.device)), "mpt_step_finish")
+
+    def grad_histogram(self):
+        """Gradients of the last step per binary16 exponent field (32 bins)."""
+        h = (ctypes.c_uint64 * 32)()
+        _check(lib().mpt_grad_histogram(self._h, ctypes.byref(h)), "mpt_grad_histogram")
+        return list(h)
 
     def stats(self):
         s = Stats()

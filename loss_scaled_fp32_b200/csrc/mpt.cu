@@ -1,7 +1,7 @@
 // mpt.cu -- host side of libmpt: the C ABI declared in include/mpt.h.
 //
 // One step = two kernel launches on the caller's stream and, for the
-// waiting call, one 112-byte read-back of the control block:
+// waiting call, one 128-byte read-back of the control block:
 //   check_kernel  (2 B/param)  overflow flag, range counts, sum of squares,
 //                              last-CTA finish -> norm, clip coefficient
 //   update_kernel (20 B/param) fused unscale/clip/decay/momentum/master/FP16,
@@ -26,7 +26,7 @@
 
 using namespace mpt;
 
-static_assert(sizeof(Ctrl) == 112, "the control block read back each step is 112 bytes");
+static_assert(sizeof(Ctrl) == 128, "the control block read back each step is 128 bytes");
 
 namespace {
 
@@ -39,8 +39,8 @@ struct Layout {
     int64_t arena_total = 0;
     std::vector<Bin> bins;
     std::vector<Seg> segs;
-    size_t off_ctrl = 0, off_partials = 0, off_ptrs = 0, off_tinfo = 0, off_bins = 0,
-           off_segs = 0, off_master = 0, off_momentum = 0, off_w16 = 0, total = 0;
+    size_t off_ctrl = 0, off_stats = 0, off_partial_rec = 0, off_partials = 0, off_ptrs = 0, off_tinfo = 0,
+           off_bins = 0, off_segs = 0, off_master = 0, off_momentum = 0, off_w16 = 0, total = 0;
 };
 
 bool config_ok(const mpt_config& c)
@@ -51,7 +51,16 @@ bool config_ok(const mpt_config& c)
         return false;
     if (!(c.min_scale > 0.0f) || !std::isfinite(c.max_scale) || !(c.max_scale >= c.min_scale))
         return false;
-    if (c.flags & ~(MPT_FLAG_CHECKED | MPT_FLAG_COUNT_STALE))
+    if (c.flags & ~(MPT_FLAG_CHECKED | MPT_FLAG_COUNT_STALE | MPT_FLAG_GRAD_STATS))
+        return false;
+    if (c.scaler_mode != MPT_SCALER_DYNAMIC && c.scaler_mode != MPT_SCALER_DIRECT)
+        return false;
+    if (!(c.direct_margin > 0.0f) || !std::isfinite(c.direct_margin))
+        return false;
+    if (c.optimizer != MPT_OPT_MOMENTUM && c.optimizer != MPT_OPT_NESTEROV &&
+        c.optimizer != MPT_OPT_ADAGRAD)
+        return false;
+    if (!(c.eps >= 0.0f) || !std::isfinite(c.eps))
         return false;
     if (c.chunk_elems != 0 && (c.chunk_elems < kChunkQuantum || c.chunk_elems > kMaxChunk ||
                                c.chunk_elems % kChunkQuantum != 0))
@@ -69,6 +78,10 @@ mpt_config defaults()
     c.max_scale = std::ldexp(1.0f, 24);
     c.flags = 0;
     c.chunk_elems = 0;
+    c.scaler_mode = MPT_SCALER_DYNAMIC;
+    c.direct_margin = 2.0f;
+    c.optimizer = MPT_OPT_MOMENTUM;
+    c.eps = 1e-10f;
     return c;
 }
 
@@ -140,6 +153,8 @@ int build_layout(const int64_t* sizes, int32_t n, int32_t chunk, Layout& L)
         return at;
     };
     L.off_ctrl = region(sizeof(Ctrl));
+    L.off_stats = region(sizeof(StatsBlock));
+    L.off_partial_rec = region(sizeof(Partial));
     L.off_partials = region(sizeof(double) * L.bins.size());
     L.off_ptrs = region(sizeof(void*) * (size_t)n);
     L.off_tinfo = region(sizeof(TensorInfo) * (size_t)n);
@@ -166,6 +181,8 @@ struct mpt_handle {
     char* ws = nullptr;
     // device views into the workspace
     Ctrl* d_ctrl = nullptr;
+    StatsBlock* d_stats = nullptr;
+    Partial* d_partial_rec = nullptr;     // this rank's record (sharded step)
     double* d_partials = nullptr;
     const uint16_t** d_ptrs = nullptr;
     TensorInfo* d_tinfo = nullptr;
@@ -180,6 +197,8 @@ struct mpt_handle {
     const void** pinned_ptrs = nullptr;  // staging of the pointer table
     cudaEvent_t ptrs_copied = nullptr;   // the last pointer-table copy is done
     Ctrl* mailbox = nullptr;             // pinned copy of the control block
+    unsigned long long* hist_box = nullptr;  // pinned copy of the histogram
+    uint64_t hist[32] = {};
     float scale = 1.0f;                  // host mirror of the device scale state
     int32_t clean_run = 0;
     mpt_stats_t stats{};
@@ -203,6 +222,8 @@ static void release(mpt_handle* h)
         cudaFreeHost(h->pinned_ptrs);
     if (h->mailbox)
         cudaFreeHost(h->mailbox);
+    if (h->hist_box)
+        cudaFreeHost(h->hist_box);
     delete h;
 }
 
@@ -223,16 +244,27 @@ static bool timing_pop(mpt_handle* h)
     return true;
 }
 
-template <bool kChecked>
+template <bool kChecked, int kStats>
 static void launch_check(const CheckArgs& a, cudaStream_t st)
 {
-    check_kernel<kChecked><<<a.t.nbins, kThreads, 0, st>>>(a);
+    check_kernel<kChecked, kStats><<<a.t.nbins, kThreads, 0, st>>>(a);
 }
+
+// Statistics the check pass gathers: the histogram with MPT_FLAG_GRAD_STATS,
+// the largest magnitude alone for the direct scaler mode.
+static int stats_level(const mpt_handle* h)
+{
+    if (h->cfg.flags & MPT_FLAG_GRAD_STATS)
+        return kMaxHist;
+    return h->cfg.scaler_mode == MPT_SCALER_DIRECT ? kMaxOnly : kNoStats;
+}
+
+static bool stats_on(const mpt_handle* h) { return stats_level(h) != kNoStats; }
 
 // The update kernel may start while the check kernel drains (programmatic
 // dependent launch): its CTAs take the SMs the check CTAs free, load their
 // work descriptors, then wait for the check result (griddepcontrol.wait).
-template <bool kStale, bool kChecked>
+template <int kOpt, bool kStale, bool kChecked>
 static void launch_update(const UpdateArgs& a, cudaStream_t st)
 {
     cudaLaunchConfig_t lc = {};
@@ -245,15 +277,57 @@ static void launch_update(const UpdateArgs& a, cudaStream_t st)
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     lc.attrs = attr;
     lc.numAttrs = 1;
-    cudaLaunchKernelEx(&lc, update_kernel<kStale, kChecked>, a);
+    cudaLaunchKernelEx(&lc, update_kernel<kOpt, kStale, kChecked>, a);
 }
 
-// Queue one step (both kernels) on st.  scale_on_device: S comes from the
-// device scale state instead of host_scale.
+template <int kOpt>
+static void launch_update_opt(const UpdateArgs& a, bool stale, bool checked, cudaStream_t st)
+{
+    if (stale)
+        checked ? launch_update<kOpt, true, true>(a, st) : launch_update<kOpt, true, false>(a, st);
+    else
+        checked ? launch_update<kOpt, false, true>(a, st) : launch_update<kOpt, false, false>(a, st);
+}
+
+static void launch_check_level(const mpt_handle* h, const CheckArgs& ca, bool checked, cudaStream_t st)
+{
+    switch (stats_level(h)) {
+    case kMaxHist:
+        checked ? launch_check<true, kMaxHist>(ca, st) : launch_check<false, kMaxHist>(ca, st);
+        break;
+    case kMaxOnly:
+        checked ? launch_check<true, kMaxOnly>(ca, st) : launch_check<false, kMaxOnly>(ca, st);
+        break;
+    default:
+        checked ? launch_check<true, kNoStats>(ca, st) : launch_check<false, kNoStats>(ca, st);
+        break;
+    }
+}
+
+static void launch_update_any(const mpt_handle* h, const UpdateArgs& ua, bool stale, bool checked,
+                              cudaStream_t st)
+{
+    switch (h->cfg.optimizer) {
+    case MPT_OPT_NESTEROV: launch_update_opt<kOptNesterov>(ua, stale, checked, st); break;
+    case MPT_OPT_ADAGRAD: launch_update_opt<kOptAdagrad>(ua, stale, checked, st); break;
+    default: launch_update_opt<kOptMomentum>(ua, stale, checked, st); break;
+    }
+}
+
+// What enqueue_step queues: the whole step, or one half of a sharded step
+// (the check pass writing this shard's record / the combine-and-finish kernel
+// followed by the update).
+enum class Phase { kWhole, kShardCheck, kShardFinish };
+
+// Queue a step (or a phase of a sharded step) on st.  scale_on_device: S
+// comes from the device scale state instead of host_scale.
 static int enqueue_step(mpt_handle* h, const void* const* d_grads_half, bool scale_on_device,
                         float host_scale, float lr, float momentum, float weight_decay,
-                        float clip, cudaStream_t st)
+                        float clip, cudaStream_t st, Phase phase = Phase::kWhole,
+                        const void* d_parts = nullptr, int32_t world = 0)
 {
+    if (phase == Phase::kShardFinish)
+        d_grads_half = h->last_ptrs.data();  // the pointers of the check pass
     for (int32_t i = 0; i < h->n; ++i) {
         const uintptr_t p = reinterpret_cast<uintptr_t>(d_grads_half[i]);
         if (p == 0 || (p & 1))
@@ -297,6 +371,10 @@ static int enqueue_step(mpt_handle* h, const void* const* d_grads_half, bool sca
     ca.scaler.growth_interval = h->cfg.growth_interval;
     ca.scaler.min_scale = h->cfg.min_scale;
     ca.scaler.max_scale = h->cfg.max_scale;
+    ca.scaler.mode = h->cfg.scaler_mode;
+    ca.scaler.direct_margin = h->cfg.direct_margin;
+    ca.stats = h->d_stats;
+    ca.partial_out = phase == Phase::kShardCheck ? h->d_partial_rec : nullptr;
 
     UpdateArgs ua;
     ua.t = t;
@@ -307,6 +385,26 @@ static int enqueue_step(mpt_handle* h, const void* const* d_grads_half, bool sca
     ua.lr = lr;
     ua.mu = momentum;
     ua.wd = weight_decay;
+    ua.eps = h->cfg.eps;
+
+    const bool checked = (h->cfg.flags & MPT_FLAG_CHECKED) != 0;
+    const bool stale = (h->cfg.flags & MPT_FLAG_COUNT_STALE) != 0;
+    if (phase != Phase::kWhole) {  // sharded step halves (not timed)
+        if (phase == Phase::kShardCheck) {
+            launch_check_level(h, ca, checked, st);
+        } else {
+            FinishArgs fa;
+            fa.parts = static_cast<const Partial*>(d_parts);
+            fa.world = world;
+            fa.have_max = stats_on(h) ? 1 : 0;
+            fa.ctrl = h->d_ctrl;
+            fa.clip = clip;
+            fa.scaler = ca.scaler;
+            finish_kernel<<<1, 32, 0, st>>>(fa);
+            launch_update_any(h, ua, stale, checked, st);
+        }
+        return cudaGetLastError() == cudaSuccess ? MPT_OK : MPT_ERR_CUDA;
+    }
 
     cudaEvent_t* ev = nullptr;
     if (h->timing) {
@@ -315,18 +413,13 @@ static int enqueue_step(mpt_handle* h, const void* const* d_grads_half, bool sca
         ev = &h->tev[3 * (int)(h->t_head % kTimingRing)];
         h->t_head += 1;
     }
-    const bool checked = (h->cfg.flags & MPT_FLAG_CHECKED) != 0;
-    const bool stale = (h->cfg.flags & MPT_FLAG_COUNT_STALE) != 0;
     bool ok = true;
     if (ev)
         ok = ok && cudaEventRecord(ev[0], st) == cudaSuccess;
-    checked ? launch_check<true>(ca, st) : launch_check<false>(ca, st);
+    launch_check_level(h, ca, checked, st);
     if (ev)
         ok = ok && cudaEventRecord(ev[1], st) == cudaSuccess;
-    if (stale)
-        checked ? launch_update<true, true>(ua, st) : launch_update<true, false>(ua, st);
-    else
-        checked ? launch_update<false, true>(ua, st) : launch_update<false, false>(ua, st);
+    launch_update_any(h, ua, stale, checked, st);
     if (ev)
         ok = ok && cudaEventRecord(ev[2], st) == cudaSuccess;
     ok = ok && cudaGetLastError() == cudaSuccess;
@@ -337,8 +430,12 @@ static int enqueue_step(mpt_handle* h, const void* const* d_grads_half, bool sca
 // state on the host and turn it into a step result.
 static int read_result(mpt_handle* h, cudaStream_t st, mpt_step_result* out)
 {
-    if (cudaMemcpyAsync(h->mailbox, h->d_ctrl, sizeof(Ctrl), cudaMemcpyDeviceToHost, st) != cudaSuccess ||
-        cudaStreamSynchronize(st) != cudaSuccess)
+    if (cudaMemcpyAsync(h->mailbox, h->d_ctrl, sizeof(Ctrl), cudaMemcpyDeviceToHost, st) != cudaSuccess)
+        return MPT_ERR_CUDA;
+    if (stats_level(h) == kMaxHist && cudaMemcpyAsync(h->hist_box, h->d_stats->hist, sizeof(h->hist),
+                                       cudaMemcpyDeviceToHost, st) != cudaSuccess)
+        return MPT_ERR_CUDA;
+    if (cudaStreamSynchronize(st) != cudaSuccess)
         return MPT_ERR_CUDA;
     while (h->t_tail < h->t_head)
         if (!timing_pop(h))
@@ -358,6 +455,11 @@ static int read_result(mpt_handle* h, cudaStream_t st, mpt_step_result* out)
     r.n_fp16_stale = stale ? c.stale_acc : 0;
     r.new_scale = c.scale;
     r.clean_run = c.clean_run;
+    if (stats_on(h))
+        r.max_abs_grad = c.max_abs;
+    if (stats_level(h) == kMaxHist)
+        for (int k = 0; k < 32; ++k)
+            h->hist[k] = h->hist_box[k];
     h->scale = c.scale;
     h->clean_run = c.clean_run;
     if (c.steps_total > h->stats.steps)
@@ -457,6 +559,8 @@ int mpt_create(const int64_t* sizes, int32_t n, const mpt_config* cfg, void* d_w
     const Layout& L = h->L;
     h->ws = ws;
     h->d_ctrl = reinterpret_cast<Ctrl*>(ws + L.off_ctrl);
+    h->d_stats = reinterpret_cast<StatsBlock*>(ws + L.off_stats);
+    h->d_partial_rec = reinterpret_cast<Partial*>(ws + L.off_partial_rec);
     h->d_partials = reinterpret_cast<double*>(ws + L.off_partials);
     h->d_ptrs = reinterpret_cast<const uint16_t**>(ws + L.off_ptrs);
     h->d_tinfo = reinterpret_cast<TensorInfo*>(ws + L.off_tinfo);
@@ -475,10 +579,12 @@ int mpt_create(const int64_t* sizes, int32_t n, const mpt_config* cfg, void* d_w
               cudaMemcpy(h->d_bins, L.bins.data(), sizeof(Bin) * L.bins.size(), cudaMemcpyHostToDevice) == cudaSuccess &&
               cudaMemcpy(h->d_segs, L.segs.data(), sizeof(Seg) * L.segs.size(), cudaMemcpyHostToDevice) == cudaSuccess &&
               cudaMemset(h->d_ctrl, 0, sizeof(Ctrl)) == cudaSuccess &&
+              cudaMemset(h->d_stats, 0, sizeof(StatsBlock)) == cudaSuccess &&
               cudaMemset(h->d_ptrs, 0, sizeof(void*) * n) == cudaSuccess &&
               cudaMemset(ws + L.off_master, 0, L.total - L.off_master) == cudaSuccess &&
               cudaHostAlloc(reinterpret_cast<void**>(&h->pinned_ptrs), sizeof(void*) * n, cudaHostAllocDefault) == cudaSuccess &&
               cudaHostAlloc(reinterpret_cast<void**>(&h->mailbox), sizeof(Ctrl), cudaHostAllocDefault) == cudaSuccess &&
+              cudaHostAlloc(reinterpret_cast<void**>(&h->hist_box), sizeof(h->hist), cudaHostAllocDefault) == cudaSuccess &&
               cudaEventCreateWithFlags(&h->ptrs_copied, cudaEventDisableTiming) == cudaSuccess &&
               upload_scaler_state(h, 1.0f, 0) &&
               cudaDeviceSynchronize() == cudaSuccess;
@@ -560,6 +666,48 @@ int mpt_step_async(mpt_handle* h, const void* const* d_grads_half, float lr, flo
     return rc == MPT_ERR_CUDA ? fail_cuda(h) : rc;
 }
 
+int mpt_shard_len(int64_t total, int32_t world, int64_t* shard_len)
+{
+    if (total <= 0 || world <= 0 || !shard_len)
+        return MPT_ERR_INVALID_ARG;
+    const int64_t per = (total + world - 1) / world;
+    *shard_len = (per + kArenaAlign - 1) / kArenaAlign * kArenaAlign;
+    return MPT_OK;
+}
+
+int mpt_step_partial(mpt_handle* h, const void* const* d_grads_half, void* cuda_stream,
+                     void** d_partial)
+{
+    if (!h || !d_grads_half || !d_partial)
+        return MPT_ERR_INVALID_ARG;
+    if (h->broken)
+        return MPT_ERR_BROKEN;
+    const int rc = enqueue_step(h, d_grads_half, true, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f,
+                                static_cast<cudaStream_t>(cuda_stream), Phase::kShardCheck);
+    if (rc == MPT_ERR_CUDA)
+        return fail_cuda(h);
+    if (rc == MPT_OK)
+        *d_partial = h->d_partial_rec;
+    return rc;
+}
+
+int mpt_step_finish(mpt_handle* h, const void* d_partials, int32_t world, float lr,
+                    float momentum, float weight_decay, float clip, void* cuda_stream)
+{
+    if (!h || !d_partials || world <= 0 || (reinterpret_cast<uintptr_t>(d_partials) & 15) != 0)
+        return MPT_ERR_INVALID_ARG;
+    if (h->broken)
+        return MPT_ERR_BROKEN;
+    if (!finite(lr) || !finite(momentum) || !finite(weight_decay) || !finite(clip))
+        return MPT_ERR_INVALID_ARG;
+    if (!h->ptrs_uploaded)
+        return MPT_ERR_INVALID_ARG;  // no check pass queued before
+    const int rc = enqueue_step(h, nullptr, true, 0.0f, lr, momentum, weight_decay, clip,
+                                static_cast<cudaStream_t>(cuda_stream), Phase::kShardFinish,
+                                d_partials, world);
+    return rc == MPT_ERR_CUDA ? fail_cuda(h) : rc;
+}
+
 int mpt_wait(mpt_handle* h, void* cuda_stream, mpt_step_result* out)
 {
     if (!h)
@@ -575,6 +723,15 @@ int mpt_device_scale(const mpt_handle* h, float** d_scale)
     if (!h || !d_scale)
         return MPT_ERR_INVALID_ARG;
     *d_scale = &h->d_ctrl->scale;
+    return MPT_OK;
+}
+
+int mpt_grad_histogram(const mpt_handle* h, uint64_t counts[32])
+{
+    if (!h || !counts)
+        return MPT_ERR_INVALID_ARG;
+    for (int k = 0; k < 32; ++k)
+        counts[k] = h->hist[k];
     return MPT_OK;
 }
 

@@ -77,6 +77,39 @@ struct __align__(16) Ctrl {
     int32_t clean_run;     // consecutive clean steps so far
     unsigned long long steps_total;
     unsigned long long skipped_total;
+    // gradient statistics (statistics mode): largest finite |g16| pattern
+    unsigned int max_mag_acc;  // accumulated by the check CTAs (atomicMax)
+    unsigned int max_mag;      // the last step's
+    float max_abs;             // its unscaled value, fp32(max|g16|) * (1/S)
+    unsigned int pad;
+};
+
+// What one rank's check pass contributes to a sharded step (32 bytes): its
+// shard's sum of squares, non-finite count and largest finite magnitude.
+// Every rank gathers all ranks' records and adds them in rank order.
+struct __align__(16) Partial {
+    double sumsq;
+    unsigned long long n_nonfinite;
+    unsigned int max_mag;
+    unsigned int error;
+    unsigned int pad[2];
+};
+
+// Histogram of binary16 exponent fields (statistics mode).
+struct __align__(16) StatsBlock {
+    unsigned long long hist_acc[32];  // accumulated by the check CTAs
+    unsigned long long hist[32];      // the last step's
+};
+
+enum Optimizer : int32_t {
+    kOptMomentum = 0,  // SGD with momentum (the pages' Step 7)
+    kOptNesterov = 1,  // Nesterov momentum
+    kOptAdagrad = 2,   // Adagrad (momentum arena holds the sum of squares)
+};
+
+enum ScalerMode : int32_t {
+    kScalerDynamic = 0,  // backoff on overflow, growth after N clean steps
+    kScalerDirect = 1,   // S = 65504 / (margin * max|g|) of each clean step
 };
 
 enum ErrorBits : unsigned int {

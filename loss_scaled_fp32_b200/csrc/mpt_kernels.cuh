@@ -36,13 +36,15 @@ struct Tables {
     int64_t arena_total;
 };
 
-// Loss-scale state machine parameters (dynamic loss scaling).
+// Loss-scale state machine parameters.
 struct ScalerParams {
     float backoff;
     float growth;
     int32_t growth_interval;
     float min_scale;
     float max_scale;
+    int32_t mode;           // kScalerDynamic or kScalerDirect
+    float direct_margin;    // direct mode: S = 65504 / (margin * max|g|)
 };
 
 struct CheckArgs {
@@ -53,6 +55,9 @@ struct CheckArgs {
     int32_t scale_on_device;  // 1: S is ctrl->scale (asynchronous steps)
     float clip;           // <= 0: off
     ScalerParams scaler;
+    StatsBlock* stats;    // statistics mode only
+    Partial* partial_out; // sharded step: write this shard's totals here and
+                          // leave the finish to finish_kernel; nullptr: finish
 };
 
 struct UpdateArgs {
@@ -64,6 +69,7 @@ struct UpdateArgs {
     float lr;
     float mu;
     float wd;
+    float eps;            // Adagrad only
 };
 
 // What the squares need from S: the binary32 reciprocal 1/S and, when S is a
@@ -85,6 +91,64 @@ __device__ __forceinline__ SqParams sq_params(float S)
     q.dscale = q.pow2 ? __longlong_as_double((long long)(1008 - e + 1023) << 52) : 0.0;
     return q;
 }
+
+// Step result and loss-scale state from the step's totals (one thread): the
+// norm, the clip coefficient, 1/S for the update, the state machine, and the
+// update kernel's counters cleared for this step.
+__device__ __forceinline__ void finish_step(Ctrl* c, float S, const SqParams& q,
+                                            unsigned long long n_nonfinite, double sumsq,
+                                            unsigned int max_mag, bool have_max,
+                                            unsigned int err, float clip, const ScalerParams& sp)
+{
+    const bool found = n_nonfinite != 0;
+    const double norm = found ? __longlong_as_double(0x7ff0000000000000ll) : sqrt(sumsq);
+    const bool clipped = !found && clip > 0.0f && norm > (double)clip;
+    float max_abs = 0.0f;
+    if (have_max) {
+        c->max_mag = max_mag;
+        max_abs = __fmul_rn(__half2float(__ushort_as_half((unsigned short)max_mag)), q.inv_scale);
+        c->max_abs = max_abs;
+    }
+    c->sumsq = sumsq;
+    c->norm = norm;
+    c->n_nonfinite = n_nonfinite;
+    c->found_inf = found ? 1 : 0;
+    c->clipped = clipped ? 1 : 0;
+    c->coef = clipped ? __double2float_rn((double)clip / norm) : 1.0f;
+    c->inv_scale = q.inv_scale;
+    c->scale_used = S;
+    c->error = err;
+    // Loss-scale state machine: on overflow skip and multiply S by beta;
+    // dynamic mode: after growth_interval consecutive clean steps multiply S
+    // by alpha; direct mode: S = 65504 / (margin * max|g|) of this step
+    // (binary64, rounded to binary32; all-zero gradients keep S).
+    int32_t clean = c->clean_run;
+    float next = S;
+    if (found) {
+        next = fmaxf(__fmul_rn(S, sp.backoff), sp.min_scale);
+        clean = 0;
+        c->skipped_total += 1;
+    } else {
+        clean += 1;
+        if (sp.mode == kScalerDirect) {
+            if (max_abs > 0.0f) {
+                const double d = __ddiv_rn(65504.0, __dmul_rn((double)sp.direct_margin,
+                                                              (double)max_abs));
+                next = fminf(fmaxf(__double2float_rn(d), sp.min_scale), sp.max_scale);
+            }
+        } else if (sp.growth_interval > 0 && clean >= sp.growth_interval) {
+            next = fminf(__fmul_rn(S, sp.growth), sp.max_scale);
+            clean = 0;
+        }
+    }
+    c->scale = next;
+    c->clean_run = clean;
+    c->steps_total += 1;
+    c->zero_acc = 0;
+    c->subnormal_acc = 0;
+    c->stale_acc = 0;
+}
+
 
 // ---------------------------------------------------------------------------
 // small helpers
@@ -214,11 +278,63 @@ __device__ __forceinline__ void sq_vec(uint2 v, const SqParams& a, SqAcc& s)
     sq_word<kPow2>(v.y, a, s);
 }
 
+// Statistics mode: each thread counts the binary16 exponent fields it sees in
+// its own row of a shared-memory table (rows padded to 33 words, so that
+// threads of a warp incrementing the same bin hit different banks) and keeps
+// the largest magnitude bit pattern.
+struct StatsAcc {
+    uint32_t* row;
+    uint32_t mx = 0;
+};
+
+// Statistics levels: kNoStats; kMaxOnly (the direct scaler mode needs only
+// the largest magnitude); kMaxHist (also the exponent histogram).
+constexpr int kNoStats = 0, kMaxOnly = 1, kMaxHist = 2;
+
+template <int kStats>
+__device__ __forceinline__ void stats_half(uint32_t h, StatsAcc* st)
+{
+    if constexpr (kStats != kNoStats) {
+        const uint32_t m = h & 0x7FFFu;
+        if constexpr (kStats == kMaxHist)
+            st->row[m >> 10] += 1;
+        st->mx = max(st->mx, m);
+    }
+}
+
+template <int kStats>
+__device__ __forceinline__ void stats_word(uint32_t w, StatsAcc* st)
+{
+    if constexpr (kStats == kMaxOnly) {
+        // both lanes at once: max of the two 15-bit magnitudes
+        st->mx = max(st->mx, max(w & 0x7FFFu, (w >> 16) & 0x7FFFu));
+    } else if constexpr (kStats == kMaxHist) {
+        stats_half<kStats>(w & 0xFFFFu, st);
+        stats_half<kStats>(w >> 16, st);
+    }
+}
+
+template <int kStats>
+__device__ __forceinline__ void stats_vec(uint4 v, StatsAcc* st)
+{
+    stats_word<kStats>(v.x, st);
+    stats_word<kStats>(v.y, st);
+    stats_word<kStats>(v.z, st);
+    stats_word<kStats>(v.w, st);
+}
+
+template <int kStats>
+__device__ __forceinline__ void stats_vec(uint2 v, StatsAcc* st)
+{
+    stats_word<kStats>(v.x, st);
+    stats_word<kStats>(v.y, st);
+}
+
 // One contiguous range: 16-B loads when aligned, 8-B when 8-B aligned, else
 // 2-B loads; unrolled so that every thread has 64 B of loads in flight.
-template <bool kPow2, typename Vec>
+template <bool kPow2, typename Vec, int kStats = kNoStats>
 __device__ __forceinline__ void check_range_vec(const uint16_t* g, int len, const SqParams& a,
-                                                SqAcc& s)
+                                                SqAcc& s, StatsAcc* st = nullptr)
 {
     constexpr int kPer = sizeof(Vec) / 2;
     constexpr int kUnroll = 64 / sizeof(Vec);
@@ -231,24 +347,32 @@ __device__ __forceinline__ void check_range_vec(const uint16_t* g, int len, cons
         for (int k = 0; k < kUnroll; ++k)
             v[k] = __ldg(gv + i + k * kThreads);
 #pragma unroll
-        for (int k = 0; k < kUnroll; ++k)
+        for (int k = 0; k < kUnroll; ++k) {
             sq_vec<kPow2>(v[k], a, s);
+            stats_vec<kStats>(v[k], st);
+        }
     }
-    for (; i < nv; i += kThreads)
-        sq_vec<kPow2>(__ldg(gv + i), a, s);
-    for (int j = nv * kPer + threadIdx.x; j < len; j += kThreads)
-        sq_half<kPow2>(__ldg(g + j), a, s);
+    for (; i < nv; i += kThreads) {
+        const Vec v = __ldg(gv + i);
+        sq_vec<kPow2>(v, a, s);
+        stats_vec<kStats>(v, st);
+    }
+    for (int j = nv * kPer + threadIdx.x; j < len; j += kThreads) {
+        const uint16_t h = __ldg(g + j);
+        sq_half<kPow2>(h, a, s);
+        stats_half<kStats>(h, st);
+    }
 }
 
-template <bool kPow2>
+template <bool kPow2, int kStats = kNoStats>
 __device__ __forceinline__ void check_range(const uint16_t* g, int len, const SqParams& a,
-                                            SqAcc& s)
+                                            SqAcc& s, StatsAcc* st = nullptr)
 {
     const uintptr_t p = reinterpret_cast<uintptr_t>(g);
     if ((p & 15) == 0) {
-        check_range_vec<kPow2, uint4>(g, len, a, s);
+        check_range_vec<kPow2, uint4, kStats>(g, len, a, s, st);
     } else if ((p & 7) == 0) {
-        check_range_vec<kPow2, uint2>(g, len, a, s);
+        check_range_vec<kPow2, uint2, kStats>(g, len, a, s, st);
     } else {
         int j = threadIdx.x;
         for (; j + 3 * kThreads < len; j += 4 * kThreads) {
@@ -257,11 +381,16 @@ __device__ __forceinline__ void check_range(const uint16_t* g, int len, const Sq
             for (int k = 0; k < 4; ++k)
                 h[k] = __ldg(g + j + k * kThreads);
 #pragma unroll
-            for (int k = 0; k < 4; ++k)
+            for (int k = 0; k < 4; ++k) {
                 sq_half<kPow2>(h[k], a, s);
+                stats_half<kStats>(h[k], st);
+            }
         }
-        for (; j < len; j += kThreads)
-            sq_half<kPow2>(__ldg(g + j), a, s);
+        for (; j < len; j += kThreads) {
+            const uint16_t h = __ldg(g + j);
+            sq_half<kPow2>(h, a, s);
+            stats_half<kStats>(h, st);
+        }
     }
 }
 
@@ -331,12 +460,46 @@ __device__ __forceinline__ void stage_packed(const Bin& bin, const Tables& t, Pa
     __syncthreads();
 }
 
-template <bool kChecked>
-__global__ void __launch_bounds__(kThreads, 8) check_kernel(CheckArgs a)
+// Largest finite |g16| bit pattern among n gradients (statistics mode, CTAs
+// that saw an inf/NaN: their running maximum included it).
+__device__ __forceinline__ uint32_t finite_max(const uint16_t* g, int n)
 {
+    uint32_t mx = 0;
+    for (int j = threadIdx.x; j < n; j += kThreads) {
+        const uint32_t m = g[j] & 0x7FFFu;
+        if (m < 0x7C00u)
+            mx = max(mx, m);
+    }
+    return mx;
+}
+
+__device__ __forceinline__ unsigned int block_max_u32(unsigned int x, unsigned int* red)
+{
+    x = __reduce_max_sync(0xffffffffu, x);
+    if ((threadIdx.x & 31) == 0)
+        red[threadIdx.x >> 5] = x;
+    __syncthreads();
+    unsigned int t = 0;
+    if (threadIdx.x == 0) {
+#pragma unroll
+        for (int w = 0; w < kWarps; ++w)
+            t = max(t, red[w]);
+    }
+    __syncthreads();
+    return t;
+}
+
+// kStats: also the largest finite |g16| and the histogram of binary16
+// exponent fields (the FP16 binades of the scaled gradients), needed by the
+// direct scaler mode and reported as statistics.
+template <bool kChecked, int kStats>
+__global__ void __launch_bounds__(kThreads, kStats == kMaxHist ? 4 : 8) check_kernel(CheckArgs a)
+{
+    constexpr int kRow = 33;  // 32 bins + 1 word of padding per thread
     __shared__ PackedStage st;
     __shared__ double s_red[kWarps];
     __shared__ unsigned int s_ured[kWarps];
+    __shared__ uint32_t s_hist[kStats == kMaxHist ? kThreads * kRow : 1];
     __shared__ int s_last;
 
     // Let the update kernel (launched with programmatic stream serialization)
@@ -352,6 +515,13 @@ __global__ void __launch_bounds__(kThreads, 8) check_kernel(CheckArgs a)
     const float S = a.scale_on_device ? a.ctrl->scale : a.host_scale;
     const SqParams q = sq_params(S);
     SqAcc s;
+    StatsAcc sa;
+    if constexpr (kStats == kMaxHist) {
+        sa.row = s_hist + threadIdx.x * kRow;
+#pragma unroll
+        for (int k = 0; k < 32; ++k)
+            sa.row[k] = 0;
+    }
     bool valid = true;
     if constexpr (kChecked)
         valid = bin_ok(bin, t);
@@ -361,19 +531,21 @@ __global__ void __launch_bounds__(kThreads, 8) check_kernel(CheckArgs a)
         if (bin.kind == kChunkBin) {
             chunk_g = t.grads[bin.tensor] + bin.tensor_begin;
             if (q.pow2)
-                check_range<true>(chunk_g, bin.n_elems, q, s);
+                check_range<true, kStats>(chunk_g, bin.n_elems, q, s, &sa);
             else
-                check_range<false>(chunk_g, bin.n_elems, q, s);
+                check_range<false, kStats>(chunk_g, bin.n_elems, q, s, &sa);
         } else {
             stage_packed(bin, t, st);
             constexpr int kU = 8;
             for (int base = 0; base < bin.n_elems; base += kU * kThreads) {
                 uint16_t h[kU];
+                bool in[kU];
 #pragma unroll
                 for (int i = 0; i < kU; ++i) {
                     const int j = base + threadIdx.x + i * kThreads;
                     h[i] = 0;  // +0: adds nothing, is finite
-                    if (j < bin.n_elems) {
+                    in[i] = j < bin.n_elems;
+                    if (in[i]) {
                         const int k = find_seg(st.begin, bin.n_segs, j);
                         h[i] = __ldg(st.gptr[k] + (j - st.begin[k]));
                     }
@@ -387,32 +559,62 @@ __global__ void __launch_bounds__(kThreads, 8) check_kernel(CheckArgs a)
                     for (int i = 0; i < kU; ++i)
                         sq_half<false>(h[i], q, s);
                 }
+                if constexpr (kStats != kNoStats) {
+#pragma unroll
+                    for (int i = 0; i < kU; ++i)
+                        if (in[i])
+                            stats_half<kStats>(h[i], &sa);
+                }
             }
         }
     }
 
-    // Non-finite count: exact, but only computed by a CTA that saw one.
+    // Non-finite count: exact, but only computed by a CTA that saw one (it
+    // also redoes its maximum over the finite gradients only).
     unsigned int nf = 0;
     if (__syncthreads_or(s.saw_nonfinite())) {
         unsigned int c = 0;
+        uint32_t mx = 0;
         if (bin.kind == kChunkBin) {
             c = count_nonfinite(chunk_g, bin.n_elems);
+            if constexpr (kStats != kNoStats)
+                mx = finite_max(chunk_g, bin.n_elems);
         } else {
             for (int j = threadIdx.x; j < bin.n_elems; j += kThreads) {
                 const int k = find_seg(st.begin, bin.n_segs, j);
-                c += ((st.gptr[k][j - st.begin[k]] & 0x7C00u) == 0x7C00u) ? 1u : 0u;
+                const uint32_t m = st.gptr[k][j - st.begin[k]] & 0x7FFFu;
+                c += m >= 0x7C00u ? 1u : 0u;
+                if (m < 0x7C00u)
+                    mx = max(mx, m);
             }
         }
+        sa.mx = mx;
         nf = block_sum_u32(c, s_ured);
     }
 
     const double part = block_sum(s.a0 + s.a1, s_red);
+    if constexpr (kStats != kNoStats) {
+        const unsigned int mx = block_max_u32(sa.mx, s_ured);   // ends with __syncthreads
+        if (kStats == kMaxHist && threadIdx.x < 32) {
+            unsigned long long n = 0;
+            for (int r = 0; r < kThreads; ++r)
+                n += s_hist[r * kRow + threadIdx.x];
+            if (n)
+                atomicAdd(&a.stats->hist_acc[threadIdx.x], n);
+            __threadfence();
+        }
+        if (threadIdx.x == 0 && mx)
+            atomicMax(&a.ctrl->max_mag_acc, mx);
+    }
     if (threadIdx.x == 0) {
         a.partials[blockIdx.x] = part;
         if (nf)
             atomicAdd(&a.ctrl->nonfinite_acc, (unsigned long long)nf);
         if (!valid)
             atomicOr(&a.ctrl->error_acc, (unsigned int)kErrBadBin);
+    }
+    __syncthreads();  // every write of this CTA precedes its ticket
+    if (threadIdx.x == 0) {
         __threadfence();
         const unsigned int ticket = atomicAdd(&a.ctrl->ticket, 1u);
         s_last = (ticket == gridDim.x - 1);
@@ -428,48 +630,60 @@ __global__ void __launch_bounds__(kThreads, 8) check_kernel(CheckArgs a)
     for (int k = threadIdx.x; k < t.nbins; k += kThreads)
         x += __ldcg(a.partials + k);
     const double sumsq = block_sum(x, s_red);
-    if (threadIdx.x == 0) {
-        Ctrl* c = a.ctrl;
-        const unsigned long long n_nonfinite = atomicAdd(&c->nonfinite_acc, 0ull);
-        const unsigned int err = atomicOr(&c->error_acc, 0u);
-        const bool found = n_nonfinite != 0;
-        const double norm = found ? __longlong_as_double(0x7ff0000000000000ll) : sqrt(sumsq);
-        const bool clipped = !found && a.clip > 0.0f && norm > (double)a.clip;
-        c->sumsq = sumsq;
-        c->norm = norm;
-        c->n_nonfinite = n_nonfinite;
-        c->found_inf = found ? 1 : 0;
-        c->clipped = clipped ? 1 : 0;
-        c->coef = clipped ? __double2float_rn((double)a.clip / norm) : 1.0f;
-        c->inv_scale = q.inv_scale;
-        c->scale_used = S;
-        c->error = err;
-        // Loss-scale state machine: on overflow skip and multiply S by beta;
-        // after growth_interval consecutive clean steps multiply S by alpha.
-        const ScalerParams& sp = a.scaler;
-        int32_t clean = c->clean_run;
-        float next = S;
-        if (found) {
-            next = fmaxf(__fmul_rn(S, sp.backoff), sp.min_scale);
-            clean = 0;
-            c->skipped_total += 1;
-        } else {
-            clean += 1;
-            if (sp.growth_interval > 0 && clean >= sp.growth_interval) {
-                next = fminf(__fmul_rn(S, sp.growth), sp.max_scale);
-                clean = 0;
-            }
+    Ctrl* c = a.ctrl;
+    if constexpr (kStats == kMaxHist) {
+        if (threadIdx.x < 32) {
+            a.stats->hist[threadIdx.x] = atomicExch(&a.stats->hist_acc[threadIdx.x], 0ull);
         }
-        c->scale = next;
-        c->clean_run = clean;
-        c->steps_total += 1;
-        c->nonfinite_acc = 0;
-        c->error_acc = 0;
-        c->zero_acc = 0;
-        c->subnormal_acc = 0;
-        c->stale_acc = 0;
-        c->ticket = 0;
     }
+    if (threadIdx.x == 0) {
+        const unsigned long long n_nonfinite = atomicExch(&c->nonfinite_acc, 0ull);
+        const unsigned int err = atomicExch(&c->error_acc, 0u);
+        const unsigned int mm = kStats != kNoStats ? atomicExch(&c->max_mag_acc, 0u) : 0u;
+        c->ticket = 0;
+        if (a.partial_out) {
+            // sharded step: the totals of this shard; finish_kernel combines
+            // every rank's record
+            Partial p{};
+            p.sumsq = sumsq;
+            p.n_nonfinite = n_nonfinite;
+            p.max_mag = mm;
+            p.error = err;
+            *a.partial_out = p;
+        } else {
+            finish_step(c, S, q, n_nonfinite, sumsq, mm, kStats != kNoStats, err, a.clip, a.scaler);
+        }
+    }
+}
+
+// Sharded step: combine the records of all ranks -- in rank order, so every
+// rank obtains bit-identical totals -- and finish the step.  One thread.
+struct FinishArgs {
+    const Partial* parts;  // world records, gathered from every rank
+    int32_t world;
+    int32_t have_max;
+    Ctrl* ctrl;
+    float clip;
+    ScalerParams scaler;
+};
+
+__global__ void finish_kernel(FinishArgs a)
+{
+    if (threadIdx.x != 0 || blockIdx.x != 0)
+        return;
+    double sumsq = 0.0;
+    unsigned long long nf = 0;
+    unsigned int mm = 0, err = 0;
+    for (int r = 0; r < a.world; ++r) {
+        const Partial p = a.parts[r];
+        sumsq += p.sumsq;
+        nf += p.n_nonfinite;
+        mm = max(mm, p.max_mag);
+        err |= p.error;
+    }
+    Ctrl* c = a.ctrl;
+    const float S = c->scale;
+    finish_step(c, S, sq_params(S), nf, sumsq, mm, a.have_max != 0, err, a.clip, a.scaler);
 }
 
 // ---------------------------------------------------------------------------
@@ -477,19 +691,32 @@ __global__ void __launch_bounds__(kThreads, 8) check_kernel(CheckArgs a)
 // ---------------------------------------------------------------------------
 
 struct UpdParams {
-    float inv_scale, coef, lr, mu, wd;
+    float inv_scale, coef, lr, mu, wd, eps;
 };
 
 // One element, each operation rounded to binary32 on its own (no FMA).
+//   momentum: v = mu*v + d;              w = w - lr*v
+//   Nesterov: v = mu*v + d;              w = w - lr*(d + mu*v)
+//   Adagrad:  v = v + d*d (sum of squares); w = w - lr*d/(sqrt(v) + eps)
+template <int kOpt>
 __device__ __forceinline__ void upd1(float g16f, float& w, float& v, const UpdParams& p)
 {
     float g = __fmul_rn(g16f, p.inv_scale);  // unscale
     g = __fmul_rn(g, p.coef);                // global-L2 clip (coef 1: exact no-op)
     const float t = __fmul_rn(p.wd, w);      // weight decay on the FP32 master
     const float d = __fadd_rn(g, t);
-    const float u = __fmul_rn(p.mu, v);      // momentum
-    v = __fadd_rn(u, d);
-    const float s = __fmul_rn(p.lr, v);      // master update
+    float step;
+    if constexpr (kOpt == kOptAdagrad) {
+        v = __fadd_rn(v, __fmul_rn(d, d));
+        step = __fdiv_rn(d, __fadd_rn(__fsqrt_rn(v), p.eps));
+    } else {
+        const float u = __fmul_rn(p.mu, v);  // momentum
+        v = __fadd_rn(u, d);
+        step = v;
+        if constexpr (kOpt == kOptNesterov)
+            step = __fadd_rn(d, __fmul_rn(p.mu, v));
+    }
+    const float s = __fmul_rn(p.lr, step);   // master update
     w = __fsub_rn(w, s);
 }
 
@@ -521,17 +748,17 @@ __device__ __forceinline__ void stale1(float w_old, float w_new, uint32_t& stale
 
 // Four elements: 8-B FP16 gradient load, 16-B master and momentum loads,
 // 16-B + 16-B + 8-B stores (every warp access is 256 B or 512 B contiguous).
-template <bool kStale>
+template <int kOpt, bool kStale>
 __device__ __forceinline__ void upd4(uint2 g, float4& w, float4& v, uint2& h, const UpdParams& p,
                                      uint32_t& stale)
 {
     const float2 g01 = __half22float2(*reinterpret_cast<const __half2*>(&g.x));
     const float2 g23 = __half22float2(*reinterpret_cast<const __half2*>(&g.y));
     const float4 w0 = w;
-    upd1(g01.x, w.x, v.x, p);
-    upd1(g01.y, w.y, v.y, p);
-    upd1(g23.x, w.z, v.z, p);
-    upd1(g23.y, w.w, v.w, p);
+    upd1<kOpt>(g01.x, w.x, v.x, p);
+    upd1<kOpt>(g01.y, w.y, v.y, p);
+    upd1<kOpt>(g23.x, w.z, v.z, p);
+    upd1<kOpt>(g23.y, w.w, v.w, p);
     h.x = h2_bits(__floats2half2_rn(w.x, w.y));
     h.y = h2_bits(__floats2half2_rn(w.z, w.w));
     stale1<kStale>(w0.x, w.x, stale);
@@ -540,20 +767,20 @@ __device__ __forceinline__ void upd4(uint2 g, float4& w, float4& v, uint2& h, co
     stale1<kStale>(w0.w, w.w, stale);
 }
 
-template <bool kStale>
+template <int kOpt, bool kStale>
 __device__ __forceinline__ void upd_scalar(uint16_t g16, float* w, float* v, uint16_t* h,
                                            const UpdParams& p, uint32_t& stale)
 {
     float wi = *w, vi = *v;
     const float w0 = wi;
-    upd1(__half2float(__ushort_as_half(g16)), wi, vi, p);
+    upd1<kOpt>(__half2float(__ushort_as_half(g16)), wi, vi, p);
     __stcs(w, wi);
     __stcs(v, vi);
     *h = __half_as_ushort(__float2half_rn(wi));
     stale1<kStale>(w0, wi, stale);
 }
 
-template <bool kStale>
+template <int kOpt, bool kStale>
 __device__ __forceinline__ void update_range(const uint16_t* g, float* w, float* v, uint16_t* h,
                                              int len, const UpdParams& p, uint32_t& nz2,
                                              uint32_t& ns2, uint32_t& stale)
@@ -578,7 +805,7 @@ __device__ __forceinline__ void update_range(const uint16_t* g, float* w, float*
             }
 #pragma unroll
             for (int k = 0; k < kUnroll; ++k) {
-                upd4<kStale>(gq[k], wq[k], vq[k], hq[k], p, stale);
+                upd4<kOpt, kStale>(gq[k], wq[k], vq[k], hq[k], p, stale);
                 count_word(gq[k].x, nz2, ns2);
                 count_word(gq[k].y, nz2, ns2);
             }
@@ -592,7 +819,7 @@ __device__ __forceinline__ void update_range(const uint16_t* g, float* w, float*
         for (; i < nq; i += kThreads) {
             uint2 gq = __ldcs(g4 + i), hq;
             float4 wq = __ldcs(w4 + i), vq = __ldcs(v4 + i);
-            upd4<kStale>(gq, wq, vq, hq, p, stale);
+            upd4<kOpt, kStale>(gq, wq, vq, hq, p, stale);
             count_word(gq.x, nz2, ns2);
             count_word(gq.y, nz2, ns2);
             __stcs(w4 + i, wq);
@@ -603,7 +830,7 @@ __device__ __forceinline__ void update_range(const uint16_t* g, float* w, float*
     }
     for (int j = start + threadIdx.x; j < len; j += kThreads) {
         const uint16_t gh = __ldcs(g + j);
-        upd_scalar<kStale>(gh, w + j, v + j, h + j, p, stale);
+        upd_scalar<kOpt, kStale>(gh, w + j, v + j, h + j, p, stale);
         count_half(gh, nz2, ns2);
     }
 }
@@ -628,7 +855,7 @@ __device__ __forceinline__ void count_range(const uint16_t* g, int len, uint32_t
         count_half(__ldcs(g + j), nz2, ns2);
 }
 
-template <bool kStale, bool kChecked>
+template <int kOpt, bool kStale, bool kChecked>
 __global__ void __launch_bounds__(kThreads) update_kernel(UpdateArgs a)
 {
     __shared__ PackedStage st;
@@ -648,7 +875,7 @@ __global__ void __launch_bounds__(kThreads) update_kernel(UpdateArgs a)
     asm volatile("griddepcontrol.wait;" ::: "memory");
     const Ctrl* c = a.ctrl;
     const bool skip = c->found_inf != 0;
-    const UpdParams p{c->inv_scale, c->coef, a.lr, a.mu, a.wd};
+    const UpdParams p{c->inv_scale, c->coef, a.lr, a.mu, a.wd, a.eps};
     uint32_t nz2 = 0, ns2 = 0, stale = 0;
 
     if (valid) {
@@ -657,7 +884,7 @@ __global__ void __launch_bounds__(kThreads) update_kernel(UpdateArgs a)
             if (skip)
                 count_range(g, bin.n_elems, nz2, ns2);
             else
-                update_range<kStale>(g, a.master + bin.arena_begin, a.momentum + bin.arena_begin,
+                update_range<kOpt, kStale>(g, a.master + bin.arena_begin, a.momentum + bin.arena_begin,
                                      a.w16 + bin.arena_begin, bin.n_elems, p, nz2, ns2, stale);
         } else {
             stage_packed(bin, t, st);
@@ -688,7 +915,7 @@ __global__ void __launch_bounds__(kThreads) update_kernel(UpdateArgs a)
                     count_half(gh[i], nz2, ns2);
                     if (!skip) {
                         const float w0 = w[i];
-                        upd1(__half2float(__ushort_as_half(gh[i])), w[i], v[i], p);
+                        upd1<kOpt>(__half2float(__ushort_as_half(gh[i])), w[i], v[i], p);
                         __stcs(a.master + e[i], w[i]);
                         __stcs(a.momentum + e[i], v[i]);
                         a.w16[e[i]] = __half_as_ushort(__float2half_rn(w[i]));

@@ -18,7 +18,8 @@ import torch
 
 import oracle
 import workloads as W
-from loss_scaled_fp32_b200 import MPT, Config
+from loss_scaled_fp32_b200 import (MPT, MPT_FLAG_GRAD_STATS, MPT_SCALER_DIRECT,
+                                   MPT_SCALER_DYNAMIC, Config)
 
 
 def ulp_diff_f32(a, b):
@@ -45,11 +46,20 @@ def ulp_diff_f16(a, b):
 class Pair:
     """GPU optimizer + oracle state over the same workload."""
 
-    def __init__(self, cfg, shifted=(), flags=0, chunk=0, master=None):
+    def __init__(self, cfg, shifted=(), flags=0, chunk=0, master=None, direct_margin=None,
+                 optimizer="momentum", eps=1e-10):
         self.cfg = cfg
         self.layout = W.GradLayout(cfg.sizes, shifted=shifted)
+        self.direct = direct_margin is not None
+        self.hist = bool(flags & MPT_FLAG_GRAD_STATS)
+        self.stats = self.hist or self.direct
         mc = Config(backoff=cfg.backoff, growth=cfg.growth, growth_interval=cfg.growth_interval,
-                    flags=flags, chunk_elems=chunk)
+                    flags=flags, chunk_elems=chunk,
+                    scaler_mode=MPT_SCALER_DIRECT if self.direct else MPT_SCALER_DYNAMIC,
+                    direct_margin=direct_margin if self.direct else 2.0,
+                    optimizer={"momentum": 0, "nesterov": 1, "adagrad": 2}[optimizer], eps=eps)
+        self.oflags = {"momentum": 0, "nesterov": oracle.NESTEROV, "adagrad": oracle.ADAGRAD}[optimizer]
+        self.eps = eps
         self.opt = MPT(cfg.sizes, mc)
         # inputs are drawn on the GPU (same integer recipe as on the CPU) and
         # copied to the host, so both sides see identical bits
@@ -60,7 +70,9 @@ class Pair:
         self.opt.set_scaler_state(cfg.scale0, 0)
         self.state = oracle.State.from_master([m.numpy() for m in master])
         self.ocfg = oracle.scaler_cfg(backoff=cfg.backoff, growth=cfg.growth,
-                                      growth_interval=cfg.growth_interval)
+                                      growth_interval=cfg.growth_interval,
+                                      mode=oracle.SCALER_DIRECT if self.direct else oracle.SCALER_DYNAMIC,
+                                      direct_margin=direct_margin if self.direct else 2.0)
         self.scale = cfg.scale0
         self.flat = torch.zeros(self.layout.total, dtype=torch.int16, device="cuda")
         self.gviews = self.layout.views(self.flat)
@@ -87,7 +99,7 @@ class Pair:
         hv = [v.numpy().view(np.uint16) for v in self.layout.views(host)]
         r = self.opt.step(gpu_grads, self.scale, cfg.lr, cfg.momentum, cfg.weight_decay, clip)
         ro = oracle.step(self.state, hv, self.scale, cfg.lr, cfg.momentum, cfg.weight_decay,
-                         clip=clip, cfg=self.ocfg, flags=0)
+                         clip=clip, cfg=self.ocfg, flags=self.oflags, eps=self.eps)
         self.compare_result(r, ro)
         self.compare_state(f"step {self.step_no}", exact=(r["clip_coef"] == ro["clip_coef"]))
         self.scale = r["new_scale"]
@@ -97,6 +109,15 @@ class Pair:
         for k in ("found_inf", "clipped", "n_zero", "n_subnormal", "n_nonfinite"):
             assert r[k] == ro[k], (self.step_no, k, r[k], ro[k])
         assert r["new_scale"] == ro["new_scale"], (self.step_no, r["new_scale"], ro["new_scale"])
+        if self.stats:
+            assert r["max_abs_grad"] == ro["max_abs"], (self.step_no, r["max_abs_grad"], ro["max_abs"])
+            hist = self.opt.grad_histogram()
+            if self.hist:
+                assert hist == ro["exp_hist"], self.step_no
+            else:
+                assert hist == [0] * 32
+        else:
+            assert r["max_abs_grad"] == 0.0
         assert r["clean_run"] == ro["new_clean_run"]
         if ro["found_inf"]:
             assert math.isinf(r["grad_norm"]) and r["clip_coef"] == 1.0

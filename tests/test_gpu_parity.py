@@ -258,3 +258,60 @@ def test_sync_and_async_steps_share_the_scale_state():
     p.compare_state("mixed", exact=True)
     p.opt.set_scaler_state(3.0, 0)             # any S, also not a power of two
     assert p.opt.device_scale().item() == 3.0
+
+
+# ---------------------------------------------------------------------------
+# gradient statistics and the direct choice of S
+# ---------------------------------------------------------------------------
+
+from loss_scaled_fp32_b200 import MPT_FLAG_GRAD_STATS  # noqa: E402
+
+
+def test_grad_statistics_ragged_unaligned_with_overflow():
+    """Largest finite |g16| (unscaled) and the exponent-field histogram, exact,
+    over packed and chunked bins, unaligned pointers and inf/NaN steps."""
+    sizes = W.configs.ragged_sizes(n=800, seed=5, log_max=15)
+    plan = {2: [(3, 0, 0x7C00), (700, 0, 0x7E00)]}
+    cfg = custom(sizes, law=("log2_uniform", -30.0, 0.0), scale0=2.0 ** 10, growth_interval=2,
+                 steps=4, injections=lambda s: plan.get(s, []))
+    p = Pair(cfg, shifted=set(range(0, 800, 5)), flags=MPT_FLAG_GRAD_STATS)
+    for _ in range(cfg.steps):
+        r, ro = p.step()
+        assert sum(ro["exp_hist"]) == sum(sizes)
+    assert any(p.opt.grad_histogram()[e] for e in range(1, 31))
+
+
+@pytest.mark.parametrize("margin", [2.0, 1.5])
+def test_direct_scaler_mode_follows_the_oracle(margin):
+    plan = {4: [(1, 2, 0xFC00)]}
+    cfg = custom([200_000, 77, 9000], law=("log2_normal", -14.0, 2.0), scale0=2.0 ** 8,
+                 steps=8, clip=0.0, injections=lambda s: plan.get(s, []))
+    p = Pair(cfg, direct_margin=margin)
+    scales = []
+    for _ in range(cfg.steps):
+        r, ro = p.step()
+        scales.append(r["new_scale"])
+    assert len(set(scales)) > 2 and scales[3] == scales[2] * 0.5     # overflow at step 4
+
+
+# ---------------------------------------------------------------------------
+# Nesterov momentum and Adagrad
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("optimizer", ["nesterov", "adagrad"])
+def test_optimizer_variants_follow_the_oracle(optimizer):
+    sizes = W.configs.ragged_sizes(n=600, seed=9, log_max=16)
+    plan = {3: [(10, 0, 0x7C00)]}
+    cfg = custom(sizes, law=("log2_uniform", -26.0, -4.0), scale0=2.0 ** 12, growth_interval=2,
+                 clip=0.2, steps=6, injections=lambda s: plan.get(s, []))
+    p = Pair(cfg, shifted=set(range(1, 600, 7)), optimizer=optimizer)
+    for _ in range(cfg.steps):
+        p.step()
+    assert p.bitexact_steps >= cfg.steps
+
+
+@pytest.mark.parametrize("optimizer", ["nesterov", "adagrad"])
+def test_optimizer_variants_gpt2_miniature(optimizer):
+    p = Pair(miniature("gpt2_medium"), optimizer=optimizer, eps=1e-8)
+    for _ in range(4):
+        p.step(clip=0.05)
