@@ -10,7 +10,7 @@ fused update kernel (unscale, global-L2 clip, weight decay, momentum, FP32
 master, FP16 copy).  The timed loop queues K steps with mpt_step_async (the
 loss scale stays on the device, as in a training loop that multiplies its loss
 by the device scalar) and waits once at the end; ``e2e`` uses the waiting
-mpt_step, which also reads the 128-byte result back every step.  The workload
+mpt_step, which also reads the 144-byte result back every step.  The workload
 is the GPT-2-medium-shaped list (292 tensors, 354 823 168 parameters, clip
 1.0): the first of the workloads at >= 100M parameters, the size the
 80%-of-HBM target is set at.  Inputs are seeded synthetic FP16 gradients (two
@@ -45,7 +45,7 @@ METRIC = "params/sec and achieved HBM GB/s (fraction of B200 peak) per optimizer
 DEFAULT_WORKLOAD = "gpt2_medium"
 BYTES_UPDATE = 20        # per parameter: read g16 2 + w 4 + v 4, write w 4 + v 4 + w16 2
 BYTES_CHECK = 2          # per parameter: read g16
-READBACK_BYTES = 128     # the control block mpt_step copies back each step
+READBACK_BYTES = 144     # the control block mpt_step copies back each step
 FALLBACK_HBM_GBS = 6650.0
 
 

@@ -190,7 +190,7 @@ int mpt_refresh_half(mpt_handle* h, void* cuda_stream);
  * by `scale` (any 2-byte alignment; contents are only read).  lr, momentum
  * and weight_decay are eta, mu and lambda; clip <= 0 disables clipping.
  * Work is queued on cuda_stream and the call waits for it (it reads the
- * 128-byte control block back).  The scale state advances from `scale`:
+ * 144-byte control block back).  The scale state advances from `scale`:
  * out->new_scale is the S for the next step.  On overflow the arenas are
  * untouched.  Errors: MPT_ERR_INVALID_ARG, MPT_ERR_CUDA,
  * MPT_ERR_DEVICE_CHECK (checked mode; the bins that passed their check were

@@ -1,7 +1,7 @@
 // mpt.cu -- host side of libmpt: the C ABI declared in include/mpt.h.
 //
 // One step = two kernel launches on the caller's stream and, for the
-// waiting call, one 128-byte read-back of the control block:
+// waiting call, one 144-byte read-back of the control block:
 //   check_kernel  (2 B/param)  overflow flag, range counts, sum of squares,
 //                              last-CTA finish -> norm, clip coefficient
 //   update_kernel (20 B/param) fused unscale/clip/decay/momentum/master/FP16,
@@ -26,7 +26,7 @@
 
 using namespace mpt;
 
-static_assert(sizeof(Ctrl) == 128, "the control block read back each step is 128 bytes");
+static_assert(sizeof(Ctrl) == 144, "the control block read back each step is 144 bytes");
 
 namespace {
 
@@ -289,6 +289,26 @@ static void launch_update_opt(const UpdateArgs& a, bool stale, bool checked, cud
         checked ? launch_update<kOpt, false, true>(a, st) : launch_update<kOpt, false, false>(a, st);
 }
 
+// What the check pass needs from S (the same values the device computes when
+// its state machine sets S): 1/S in binary32 and, for S = 2^e with
+// -15 <= e <= 100, the binary64 constant 2^(1008-e).
+struct HostScale {
+    float inv;
+    double dscale;
+    int32_t pow2;
+};
+
+static HostScale host_scale_params(float S)
+{
+    HostScale r;
+    r.inv = 1.0f / S;
+    int e2 = 0;
+    const bool pow2 = std::frexp(S, &e2) == 0.5f && (e2 - 1) >= -15 && (e2 - 1) <= 100;
+    r.pow2 = pow2 ? 1 : 0;
+    r.dscale = pow2 ? std::ldexp(1.0, 1008 - (e2 - 1)) : 0.0;
+    return r;
+}
+
 static void launch_check_level(const mpt_handle* h, const CheckArgs& ca, bool checked, cudaStream_t st)
 {
     switch (stats_level(h)) {
@@ -364,6 +384,12 @@ static int enqueue_step(mpt_handle* h, const void* const* d_grads_half, bool sca
     ca.partials = h->d_partials;
     ca.ctrl = h->d_ctrl;
     ca.host_scale = host_scale;
+    {
+        const HostScale hp = host_scale_params(scale_on_device ? 1.0f : host_scale);
+        ca.host_inv = hp.inv;
+        ca.host_dscale = hp.dscale;
+        ca.host_pow2 = hp.pow2;
+    }
     ca.scale_on_device = scale_on_device ? 1 : 0;
     ca.clip = clip;
     ca.scaler.backoff = h->cfg.backoff;
@@ -484,14 +510,13 @@ static int fail_cuda(mpt_handle* h)
 
 static bool upload_scaler_state(mpt_handle* h, float scale, int32_t clean_run)
 {
-    struct {
-        float scale;
-        int32_t clean_run;
-    } v{scale, clean_run};
-    static_assert(offsetof(Ctrl, clean_run) == offsetof(Ctrl, scale) + sizeof(float),
-                  "scale and clean_run are adjacent");
-    return cudaMemcpy(reinterpret_cast<char*>(h->d_ctrl) + offsetof(Ctrl, scale), &v, sizeof v,
-                      cudaMemcpyHostToDevice) == cudaSuccess;
+    const HostScale p = host_scale_params(scale);
+    char* c = reinterpret_cast<char*>(h->d_ctrl);
+    return cudaMemcpy(c + offsetof(Ctrl, scale), &scale, sizeof scale, cudaMemcpyHostToDevice) == cudaSuccess &&
+           cudaMemcpy(c + offsetof(Ctrl, clean_run), &clean_run, sizeof clean_run, cudaMemcpyHostToDevice) == cudaSuccess &&
+           cudaMemcpy(c + offsetof(Ctrl, next_inv), &p.inv, sizeof p.inv, cudaMemcpyHostToDevice) == cudaSuccess &&
+           cudaMemcpy(c + offsetof(Ctrl, next_dscale), &p.dscale, sizeof p.dscale, cudaMemcpyHostToDevice) == cudaSuccess &&
+           cudaMemcpy(c + offsetof(Ctrl, next_pow2), &p.pow2, sizeof p.pow2, cudaMemcpyHostToDevice) == cudaSuccess;
 }
 
 extern "C" {

@@ -81,6 +81,11 @@ struct __align__(16) Ctrl {
     unsigned int max_mag_acc;  // accumulated by the check CTAs (atomicMax)
     unsigned int max_mag;      // the last step's
     float max_abs;             // its unscaled value, fp32(max|g16|) * (1/S)
+    // what the next check pass needs from `scale`, computed once when the
+    // state is set (1/S and, for S = 2^e with -15 <= e <= 100, 2^(1008-e))
+    int32_t next_pow2;
+    double next_dscale;
+    float next_inv;
     unsigned int pad;
 };
 

@@ -51,7 +51,10 @@ struct CheckArgs {
     Tables t;
     double* partials;     // one binary64 partial sum of squares per bin
     Ctrl* ctrl;
-    float host_scale;     // S the gradients carry, when given by the host
+    float host_scale;     // S the gradients carry, when given by the host,
+    float host_inv;       // with its binary32 reciprocal
+    double host_dscale;   // and 2^(1008-e) when S = 2^e, -15 <= e <= 100
+    int32_t host_pow2;
     int32_t scale_on_device;  // 1: S is ctrl->scale (asynchronous steps)
     float clip;           // <= 0: off
     ScalerParams scaler;
@@ -142,6 +145,10 @@ __device__ __forceinline__ void finish_step(Ctrl* c, float S, const SqParams& q,
         }
     }
     c->scale = next;
+    const SqParams nq = sq_params(next);
+    c->next_inv = nq.inv_scale;
+    c->next_dscale = nq.dscale;
+    c->next_pow2 = nq.pow2 ? 1 : 0;
     c->clean_run = clean;
     c->steps_total += 1;
     c->zero_acc = 0;
@@ -512,8 +519,20 @@ __global__ void __launch_bounds__(kThreads, kStats == kMaxHist ? 4 : 8) check_ke
     // S of these gradients: the host's, or the device state the previous
     // step left (it changes only in this kernel's last CTA, after every other
     // CTA has finished reading it)
-    const float S = a.scale_on_device ? a.ctrl->scale : a.host_scale;
-    const SqParams q = sq_params(S);
+    float S;
+    SqParams q;
+    if (a.scale_on_device) {
+        const Ctrl* c = a.ctrl;
+        S = c->scale;
+        q.inv_scale = c->next_inv;
+        q.dscale = c->next_dscale;
+        q.pow2 = c->next_pow2 != 0;
+    } else {
+        S = a.host_scale;
+        q.inv_scale = a.host_inv;
+        q.dscale = a.host_dscale;
+        q.pow2 = a.host_pow2 != 0;
+    }
     SqAcc s;
     StatsAcc sa;
     if constexpr (kStats == kMaxHist) {
@@ -682,8 +701,11 @@ __global__ void finish_kernel(FinishArgs a)
         err |= p.error;
     }
     Ctrl* c = a.ctrl;
-    const float S = c->scale;
-    finish_step(c, S, sq_params(S), nf, sumsq, mm, a.have_max != 0, err, a.clip, a.scaler);
+    SqParams q;
+    q.inv_scale = c->next_inv;
+    q.dscale = c->next_dscale;
+    q.pow2 = c->next_pow2 != 0;
+    finish_step(c, c->scale, q, nf, sumsq, mm, a.have_max != 0, err, a.clip, a.scaler);
 }
 
 // ---------------------------------------------------------------------------
@@ -693,6 +715,17 @@ __global__ void finish_kernel(FinishArgs a)
 struct UpdParams {
     float inv_scale, coef, lr, mu, wd, eps;
 };
+
+// Elements of a chunk bin whose master, momentum and gradients the update
+// kernel prefetches into L2 before it waits for the check result.
+constexpr int kPrefetchElems = 8192;
+
+// Bulk prefetch of [p, p + bytes) into L2 (non-multicast TMA; p 16-byte
+// aligned, bytes a multiple of 16, both in bounds).
+__device__ __forceinline__ void prefetch_l2(const void* p, uint32_t bytes)
+{
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+}
 
 // One element, each operation rounded to binary32 on its own (no FMA).
 //   momentum: v = mu*v + d;              w = w - lr*v
@@ -870,6 +903,19 @@ __global__ void __launch_bounds__(kThreads) update_kernel(UpdateArgs a)
     if constexpr (kChecked)
         valid = bin_ok(bin, t);
 
+    // While the check kernel drains, start this CTA's first reads: a bulk
+    // (TMA) prefetch of the start of its master, momentum and gradient ranges
+    // into L2.  They do not depend on the check result.
+    if (valid && bin.kind == kChunkBin && threadIdx.x == 0) {
+        const int n_pre = min(bin.n_elems, kPrefetchElems) & ~7;
+        if (n_pre > 0) {
+            prefetch_l2(a.master + bin.arena_begin, (uint32_t)n_pre * 4u);
+            prefetch_l2(a.momentum + bin.arena_begin, (uint32_t)n_pre * 4u);
+            const uint16_t* g = t.grads[bin.tensor] + bin.tensor_begin;
+            if ((reinterpret_cast<uintptr_t>(g) & 15) == 0)
+                prefetch_l2(g, (uint32_t)n_pre * 2u);
+        }
+    }
     // Wait until the check kernel has finished and its result is visible
     // (returns at once when this grid was launched without overlap).
     asm volatile("griddepcontrol.wait;" ::: "memory");
