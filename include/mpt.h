@@ -99,13 +99,16 @@ typedef struct {
     float min_scale;          /* lower bound of S after a backoff (2^-24)          */
     float max_scale;          /* upper bound of S after a growth (2^24)            */
     uint32_t flags;           /* MPT_FLAG_* (default 0)                            */
-    int32_t chunk_elems;      /* elements per work bin: a multiple of 2048 in
-                                 [2048, 2^20]; 0 = default (32768)                 */
+    int32_t check_chunk_elems;  /* elements per work bin (one CTA) of the check
+                                   pass: a multiple of 2048 in [2048, 2^20];
+                                   0 = default (65536)                            */
     int32_t scaler_mode;      /* MPT_SCALER_DYNAMIC (default) or _DIRECT           */
     float direct_margin;      /* direct mode: margin > 0 (default 2: one bit of
                                  headroom, as the pages suggest)                   */
     int32_t optimizer;        /* MPT_OPT_MOMENTUM (default), _NESTEROV, _ADAGRAD   */
     float eps;                /* Adagrad denominator term (default 1e-10)          */
+    int32_t update_chunk_elems; /* the same for the update pass; 0 = default
+                                   (4096)                                         */
 } mpt_config;
 
 /* ---- results ------------------------------------------------------------ */

@@ -53,9 +53,9 @@ class Config(ctypes.Structure):
     _fields_ = [("backoff", ctypes.c_float), ("growth", ctypes.c_float),
                 ("growth_interval", ctypes.c_int32), ("min_scale", ctypes.c_float),
                 ("max_scale", ctypes.c_float), ("flags", ctypes.c_uint32),
-                ("chunk_elems", ctypes.c_int32), ("scaler_mode", ctypes.c_int32),
+                ("check_chunk_elems", ctypes.c_int32), ("scaler_mode", ctypes.c_int32),
                 ("direct_margin", ctypes.c_float), ("optimizer", ctypes.c_int32),
-                ("eps", ctypes.c_float)]
+                ("eps", ctypes.c_float), ("update_chunk_elems", ctypes.c_int32)]
 
     def __init__(self, **kw):
         super().__init__()

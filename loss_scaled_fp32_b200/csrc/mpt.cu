@@ -37,10 +37,12 @@ size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 struct Layout {
     std::vector<int64_t> arena_off;
     int64_t arena_total = 0;
-    std::vector<Bin> bins;
+    std::vector<Bin> bins_check;   // work of the check pass (one CTA each)
+    std::vector<Bin> bins_update;  // work of the update pass
     std::vector<Seg> segs;
-    size_t off_ctrl = 0, off_stats = 0, off_partial_rec = 0, off_partials = 0, off_ptrs = 0, off_tinfo = 0,
-           off_bins = 0, off_segs = 0, off_master = 0, off_momentum = 0, off_w16 = 0, total = 0;
+    size_t off_ctrl = 0, off_stats = 0, off_partial_rec = 0, off_partials = 0, off_ptrs = 0,
+           off_tinfo = 0, off_bins_check = 0, off_bins_update = 0, off_segs = 0, off_master = 0,
+           off_momentum = 0, off_w16 = 0, total = 0;
 };
 
 bool config_ok(const mpt_config& c)
@@ -62,9 +64,9 @@ bool config_ok(const mpt_config& c)
         return false;
     if (!(c.eps >= 0.0f) || !std::isfinite(c.eps))
         return false;
-    if (c.chunk_elems != 0 && (c.chunk_elems < kChunkQuantum || c.chunk_elems > kMaxChunk ||
-                               c.chunk_elems % kChunkQuantum != 0))
-        return false;
+    for (int32_t ch : {c.check_chunk_elems, c.update_chunk_elems})
+        if (ch != 0 && (ch < kChunkQuantum || ch > kMaxChunk || ch % kChunkQuantum != 0))
+            return false;
     return true;
 }
 
@@ -77,7 +79,8 @@ mpt_config defaults()
     c.min_scale = std::ldexp(1.0f, -24);
     c.max_scale = std::ldexp(1.0f, 24);
     c.flags = 0;
-    c.chunk_elems = 0;
+    c.check_chunk_elems = 0;
+    c.update_chunk_elems = 0;
     c.scaler_mode = MPT_SCALER_DYNAMIC;
     c.direct_margin = 2.0f;
     c.optimizer = MPT_OPT_MOMENTUM;
@@ -85,22 +88,16 @@ mpt_config defaults()
     return c;
 }
 
-// Arena offsets (16-element aligned) and the work bins: every tensor larger
-// than kSmallTensor is cut into chunk-sized ranges, one bin each; the small
-// tensors are packed, in list order, into bins of at most kPackedMaxElems
-// elements and kMaxPackedSegs tensors.
-int build_layout(const int64_t* sizes, int32_t n, int32_t chunk, Layout& L)
+// Arena offsets (16-element aligned) and the work bins.  Every tensor larger
+// than kSmallTensor is cut into chunk-sized ranges, one bin (one CTA) each;
+// the small tensors are packed, in list order, into bins of at most
+// kPackedMaxElems elements and kMaxPackedSegs tensors.  The two kernels get
+// their own chunk size: the check pass (2 B/param, short-lived CTAs) wants
+// large bins to amortise each CTA's prologue and finish, the update pass
+// (20 B/param) small bins that keep every SM streaming to the end.
+static void chunk_bins(const int64_t* sizes, int32_t n, int32_t chunk, const Layout& L,
+                       std::vector<Bin>& out)
 {
-    L.arena_off.resize(n);
-    int64_t off = 0;
-    for (int32_t i = 0; i < n; ++i) {
-        if (sizes[i] <= 0)
-            return MPT_ERR_INVALID_ARG;
-        L.arena_off[i] = off;
-        off += (sizes[i] + kArenaAlign - 1) / kArenaAlign * kArenaAlign;
-    }
-    L.arena_total = off;
-
     for (int32_t i = 0; i < n; ++i) {
         if (sizes[i] <= kSmallTensor)
             continue;
@@ -112,9 +109,27 @@ int build_layout(const int64_t* sizes, int32_t n, int32_t chunk, Layout& L)
             b.n_elems = (int32_t)std::min<int64_t>(chunk, sizes[i] - c);
             b.n_segs = 0;
             b.kind = kChunkBin;
-            L.bins.push_back(b);
+            out.push_back(b);
         }
     }
+}
+
+int build_layout(const int64_t* sizes, int32_t n, int32_t check_chunk, int32_t update_chunk,
+                 Layout& L)
+{
+    L.arena_off.resize(n);
+    int64_t off = 0;
+    for (int32_t i = 0; i < n; ++i) {
+        if (sizes[i] <= 0)
+            return MPT_ERR_INVALID_ARG;
+        L.arena_off[i] = off;
+        off += (sizes[i] + kArenaAlign - 1) / kArenaAlign * kArenaAlign;
+    }
+    L.arena_total = off;
+
+    chunk_bins(sizes, n, check_chunk, L, L.bins_check);
+    chunk_bins(sizes, n, update_chunk, L, L.bins_update);
+    std::vector<Bin> packed;
     Bin open{};
     bool have_open = false;
     for (int32_t i = 0; i < n; ++i) {
@@ -122,7 +137,7 @@ int build_layout(const int64_t* sizes, int32_t n, int32_t chunk, Layout& L)
             continue;
         const int32_t len = (int32_t)sizes[i];
         if (have_open && (open.n_elems + len > kPackedMaxElems || open.n_segs == kMaxPackedSegs)) {
-            L.bins.push_back(open);
+            packed.push_back(open);
             have_open = false;
         }
         if (!have_open) {
@@ -142,8 +157,11 @@ int build_layout(const int64_t* sizes, int32_t n, int32_t chunk, Layout& L)
         open.n_elems += len;
     }
     if (have_open)
-        L.bins.push_back(open);
-    if (L.bins.size() > 0x7fffffffu || L.segs.size() > 0x7fffffffu)
+        packed.push_back(open);
+    L.bins_check.insert(L.bins_check.end(), packed.begin(), packed.end());
+    L.bins_update.insert(L.bins_update.end(), packed.begin(), packed.end());
+    if (L.bins_check.size() > 0x7fffffffu || L.bins_update.size() > 0x7fffffffu ||
+        L.segs.size() > 0x7fffffffu)
         return MPT_ERR_INVALID_ARG;
 
     size_t p = 0;
@@ -155,10 +173,11 @@ int build_layout(const int64_t* sizes, int32_t n, int32_t chunk, Layout& L)
     L.off_ctrl = region(sizeof(Ctrl));
     L.off_stats = region(sizeof(StatsBlock));
     L.off_partial_rec = region(sizeof(Partial));
-    L.off_partials = region(sizeof(double) * L.bins.size());
+    L.off_partials = region(sizeof(double) * L.bins_check.size());
     L.off_ptrs = region(sizeof(void*) * (size_t)n);
     L.off_tinfo = region(sizeof(TensorInfo) * (size_t)n);
-    L.off_bins = region(sizeof(Bin) * L.bins.size());
+    L.off_bins_check = region(sizeof(Bin) * L.bins_check.size());
+    L.off_bins_update = region(sizeof(Bin) * L.bins_update.size());
     L.off_segs = region(sizeof(Seg) * L.segs.size());
     L.off_master = region(sizeof(float) * (size_t)L.arena_total);
     L.off_momentum = region(sizeof(float) * (size_t)L.arena_total);
@@ -168,6 +187,9 @@ int build_layout(const int64_t* sizes, int32_t n, int32_t chunk, Layout& L)
 }
 
 bool finite(float x) { return std::isfinite(x); }
+
+int32_t check_chunk(const mpt_config& c) { return c.check_chunk_elems ? c.check_chunk_elems : kDefaultCheckChunk; }
+int32_t update_chunk(const mpt_config& c) { return c.update_chunk_elems ? c.update_chunk_elems : kDefaultUpdateChunk; }
 
 }  // namespace
 
@@ -186,7 +208,8 @@ struct mpt_handle {
     double* d_partials = nullptr;
     const uint16_t** d_ptrs = nullptr;
     TensorInfo* d_tinfo = nullptr;
-    Bin* d_bins = nullptr;
+    Bin* d_bins_check = nullptr;
+    Bin* d_bins_update = nullptr;
     Seg* d_segs = nullptr;
     float* d_master = nullptr;
     float* d_momentum = nullptr;
@@ -369,11 +392,11 @@ static int enqueue_step(mpt_handle* h, const void* const* d_grads_half, bool sca
     }
 
     Tables t;
-    t.bins = h->d_bins;
+    t.bins = h->d_bins_check;
     t.segs = h->d_segs;
     t.tensors = h->d_tinfo;
     t.grads = h->d_ptrs;
-    t.nbins = (int32_t)h->L.bins.size();
+    t.nbins = (int32_t)h->L.bins_check.size();
     t.nsegs = (int32_t)h->L.segs.size();
     t.ntensors = h->n;
     t.pad = 0;
@@ -404,6 +427,8 @@ static int enqueue_step(mpt_handle* h, const void* const* d_grads_half, bool sca
 
     UpdateArgs ua;
     ua.t = t;
+    ua.t.bins = h->d_bins_update;
+    ua.t.nbins = (int32_t)h->L.bins_update.size();
     ua.master = h->d_master;
     ua.momentum = h->d_momentum;
     ua.w16 = h->d_w16;
@@ -537,7 +562,7 @@ int mpt_workspace_bytes(const int64_t* sizes, int32_t n, const mpt_config* cfg, 
     if (!config_ok(c))
         return MPT_ERR_INVALID_ARG;
     Layout L;
-    const int rc = build_layout(sizes, n, c.chunk_elems ? c.chunk_elems : kDefaultChunk, L);
+    const int rc = build_layout(sizes, n, check_chunk(c), update_chunk(c), L);
     if (rc != MPT_OK)
         return rc;
     *bytes = L.total;
@@ -558,7 +583,7 @@ int mpt_create(const int64_t* sizes, int32_t n, const mpt_config* cfg, void* d_w
         return MPT_ERR_INVALID_ARG;
     h->cfg = c;
     h->n = n;
-    int rc = build_layout(sizes, n, c.chunk_elems ? c.chunk_elems : kDefaultChunk, h->L);
+    int rc = build_layout(sizes, n, check_chunk(c), update_chunk(c), h->L);
     if (rc != MPT_OK) {
         release(h);
         return rc;
@@ -589,7 +614,8 @@ int mpt_create(const int64_t* sizes, int32_t n, const mpt_config* cfg, void* d_w
     h->d_partials = reinterpret_cast<double*>(ws + L.off_partials);
     h->d_ptrs = reinterpret_cast<const uint16_t**>(ws + L.off_ptrs);
     h->d_tinfo = reinterpret_cast<TensorInfo*>(ws + L.off_tinfo);
-    h->d_bins = reinterpret_cast<Bin*>(ws + L.off_bins);
+    h->d_bins_check = reinterpret_cast<Bin*>(ws + L.off_bins_check);
+    h->d_bins_update = reinterpret_cast<Bin*>(ws + L.off_bins_update);
     h->d_segs = reinterpret_cast<Seg*>(ws + L.off_segs);
     h->d_master = reinterpret_cast<float*>(ws + L.off_master);
     h->d_momentum = reinterpret_cast<float*>(ws + L.off_momentum);
@@ -601,7 +627,8 @@ int mpt_create(const int64_t* sizes, int32_t n, const mpt_config* cfg, void* d_w
         tinfo[i].arena_off = L.arena_off[i];
     }
     bool ok = cudaMemcpy(h->d_tinfo, tinfo.data(), sizeof(TensorInfo) * n, cudaMemcpyHostToDevice) == cudaSuccess &&
-              cudaMemcpy(h->d_bins, L.bins.data(), sizeof(Bin) * L.bins.size(), cudaMemcpyHostToDevice) == cudaSuccess &&
+              cudaMemcpy(h->d_bins_check, L.bins_check.data(), sizeof(Bin) * L.bins_check.size(), cudaMemcpyHostToDevice) == cudaSuccess &&
+              cudaMemcpy(h->d_bins_update, L.bins_update.data(), sizeof(Bin) * L.bins_update.size(), cudaMemcpyHostToDevice) == cudaSuccess &&
               cudaMemcpy(h->d_segs, L.segs.data(), sizeof(Seg) * L.segs.size(), cudaMemcpyHostToDevice) == cudaSuccess &&
               cudaMemset(h->d_ctrl, 0, sizeof(Ctrl)) == cudaSuccess &&
               cudaMemset(h->d_stats, 0, sizeof(StatsBlock)) == cudaSuccess &&
@@ -848,7 +875,7 @@ const char* mpt_error_string(int code)
 
 namespace {
 
-constexpr int kNoAllocChunk = kDefaultChunk;
+constexpr int kNoAllocChunk = 32768;
 constexpr int64_t kNoAllocMaxBins = MPT_NOALLOC_MAX_ELEMS / kNoAllocChunk;
 constexpr size_t kNoAllocCtrlBytes = 256;
 constexpr size_t kNoAllocScratchBytes = kNoAllocCtrlBytes + sizeof(double) * kNoAllocMaxBins;

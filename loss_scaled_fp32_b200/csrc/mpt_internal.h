@@ -9,7 +9,8 @@ namespace mpt {
 constexpr int kThreads = 256;              // threads per CTA of every kernel
 constexpr int kWarps = kThreads / 32;
 constexpr int kArenaAlign = 16;            // elements: 64 B FP32, 32 B FP16
-constexpr int kDefaultChunk = 32768;       // elements per work bin
+constexpr int kDefaultCheckChunk = 65536;  // elements per check-pass bin
+constexpr int kDefaultUpdateChunk = 4096;  // elements per update-pass bin
 constexpr int kChunkQuantum = 2048;        // chunk sizes are multiples of this
 constexpr int kMaxChunk = 1 << 20;
 constexpr int kSmallTensor = 1024;         // tensors up to this size are packed

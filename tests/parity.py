@@ -54,7 +54,7 @@ class Pair:
         self.hist = bool(flags & MPT_FLAG_GRAD_STATS)
         self.stats = self.hist or self.direct
         mc = Config(backoff=cfg.backoff, growth=cfg.growth, growth_interval=cfg.growth_interval,
-                    flags=flags, chunk_elems=chunk,
+                    flags=flags, check_chunk_elems=chunk, update_chunk_elems=chunk,
                     scaler_mode=MPT_SCALER_DIRECT if self.direct else MPT_SCALER_DYNAMIC,
                     direct_margin=direct_margin if self.direct else 2.0,
                     optimizer={"momentum": 0, "nesterov": 1, "adagrad": 2}[optimizer], eps=eps)

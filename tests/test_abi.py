@@ -45,11 +45,13 @@ def test_library_builds_and_exports_every_declared_symbol():
 def test_defaults_and_config_validation():
     c = lsf.Config()
     assert (c.backoff, c.growth, c.growth_interval) == (0.5, 2.0, 0)
-    assert (c.min_scale, c.max_scale, c.flags, c.chunk_elems) == (2.0 ** -24, 2.0 ** 24, 0, 0)
+    assert (c.min_scale, c.max_scale, c.flags) == (2.0 ** -24, 2.0 ** 24, 0)
+    assert (c.check_chunk_elems, c.update_chunk_elems) == (0, 0)
     L = lsf.lib()
     sizes = (ctypes.c_int64 * 2)(10, 20)
     nb = ctypes.c_size_t()
-    for bad in (dict(chunk_elems=1000), dict(chunk_elems=1 << 21), dict(backoff=0.0),
+    for bad in (dict(check_chunk_elems=1000), dict(check_chunk_elems=1 << 21),
+                dict(update_chunk_elems=3000), dict(backoff=0.0),
                 dict(backoff=1.5), dict(growth=0.5), dict(growth_interval=-1),
                 dict(min_scale=0.0), dict(flags=0x100), dict(min_scale=4.0, max_scale=2.0)):
         assert L.mpt_workspace_bytes(sizes, 2, ctypes.byref(lsf.Config(**bad)),
@@ -78,7 +80,8 @@ def test_workspace_bytes():
     arr = (ctypes.c_int64 * 1)(5)
     assert L.mpt_workspace_bytes(arr, 0, None, ctypes.byref(ctypes.c_size_t())) == lsf.MPT_ERR_INVALID_ARG
     # smaller chunks mean more bins, hence more table bytes, never fewer
-    assert ws([10_000_000], chunk_elems=2048)[1] > ws([10_000_000])[1]
+    assert ws([10_000_000], update_chunk_elems=2048)[1] > ws([10_000_000])[1]
+    assert ws([10_000_000], check_chunk_elems=2048)[1] > ws([10_000_000])[1]
 
 
 def test_invalid_handles_and_arguments_return_codes():
