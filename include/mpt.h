@@ -101,7 +101,8 @@ typedef struct {
     uint32_t flags;           /* MPT_FLAG_* (default 0)                            */
     int32_t check_chunk_elems;  /* elements per work bin (one CTA) of the check
                                    pass: a multiple of 2048 in [2048, 2^20];
-                                   0 = default (65536)                            */
+                                   0 = default: 65536, halved down to 2048
+                                   while the list gives fewer than 2048 bins */
     int32_t scaler_mode;      /* MPT_SCALER_DYNAMIC (default) or _DIRECT           */
     float direct_margin;      /* direct mode: margin > 0 (default 2: one bit of
                                  headroom, as the pages suggest)                   */
@@ -193,7 +194,7 @@ int mpt_refresh_half(mpt_handle* h, void* cuda_stream);
  * by `scale` (any 2-byte alignment; contents are only read).  lr, momentum
  * and weight_decay are eta, mu and lambda; clip <= 0 disables clipping.
  * Work is queued on cuda_stream and the call waits for it (it reads the
- * 144-byte control block back).  The scale state advances from `scale`:
+ * 384-byte control block back).  The scale state advances from `scale`:
  * out->new_scale is the S for the next step.  On overflow the arenas are
  * untouched.  Errors: MPT_ERR_INVALID_ARG, MPT_ERR_CUDA,
  * MPT_ERR_DEVICE_CHECK (checked mode; the bins that passed their check were
@@ -290,11 +291,18 @@ int mpt_stats(const mpt_handle* h, mpt_stats_t* out);
 int mpt_get_scaler_state(const mpt_handle* h, float* scale, int32_t* clean_run);
 int mpt_set_scaler_state(mpt_handle* h, float scale, int32_t clean_run);
 
-/* Time both kernels of every following step with CUDA events recorded on the
- * step's stream (summed into mpt_stats_t at the next waiting call, or when
- * 256 timed steps are pending); enable = 0 turns it off (and waits for the
- * pending events).  Errors: MPT_ERR_INVALID_ARG, MPT_ERR_CUDA. */
-int mpt_set_timing(mpt_handle* h, int32_t enable);
+/* Time both kernels of every `every`-th following step (the first step
+ * queued after the call, then every `every`-th; 1 = every step) with CUDA
+ * events recorded on the step's stream before the check kernel, between the
+ * two kernels and after the update kernel.  The durations are summed into
+ * mpt_stats_t at the next waiting call, or when 256 timed steps are pending.
+ * The events cost time of their own (the update of a timed step cannot start
+ * early, and three more stream operations sit in each timed step), so a
+ * throughput measurement should sample: every = 10 keeps that cost to a
+ * tenth.  every = 0 turns timing off (and waits for the pending events).
+ * Whole steps only: the halves of a sharded step are not timed.
+ * Errors: MPT_ERR_INVALID_ARG (h NULL, every < 0), MPT_ERR_CUDA. */
+int mpt_set_timing(mpt_handle* h, int32_t every);
 
 /* Release the handle's host resources.  The workspace is the caller's and is
  * not freed.  NULL is accepted. */

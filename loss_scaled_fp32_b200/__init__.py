@@ -317,8 +317,10 @@ class MPT:
     def set_scaler_state(self, scale, clean_run=0):
         _check(lib().mpt_set_scaler_state(self._h, scale, clean_run), "mpt_set_scaler_state")
 
-    def set_timing(self, enable=True):
-        _check(lib().mpt_set_timing(self._h, 1 if enable else 0), "mpt_set_timing")
+    def set_timing(self, every=1):
+        """Time the two kernels of every ``every``-th following step (0 or
+        False: off; True or 1: every step)."""
+        _check(lib().mpt_set_timing(self._h, int(every)), "mpt_set_timing")
 
     def close(self):
         if getattr(self, "_h", None):

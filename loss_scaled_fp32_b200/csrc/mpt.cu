@@ -1,7 +1,7 @@
 // mpt.cu -- host side of libmpt: the C ABI declared in include/mpt.h.
 //
 // One step = two kernel launches on the caller's stream and, for the
-// waiting call, one 144-byte read-back of the control block:
+// waiting call, one 384-byte read-back of the control block:
 //   check_kernel  (2 B/param)  overflow flag, range counts, sum of squares,
 //                              last-CTA finish -> norm, clip coefficient
 //   update_kernel (20 B/param) fused unscale/clip/decay/momentum/master/FP16,
@@ -26,7 +26,9 @@
 
 using namespace mpt;
 
-static_assert(sizeof(Ctrl) == 144, "the control block read back each step is 144 bytes");
+static_assert(sizeof(Ctrl) == 384, "the control block read back each step is 384 bytes");
+static_assert(offsetof(Ctrl, zero_acc) == 128 && offsetof(Ctrl, sumsq) == 256,
+              "one 128-byte line per group of control fields");
 
 namespace {
 
@@ -40,7 +42,8 @@ struct Layout {
     std::vector<Bin> bins_check;   // work of the check pass (one CTA each)
     std::vector<Bin> bins_update;  // work of the update pass
     std::vector<Seg> segs;
-    size_t off_ctrl = 0, off_stats = 0, off_partial_rec = 0, off_partials = 0, off_ptrs = 0,
+    size_t off_ctrl = 0, off_stats = 0, off_partial_rec = 0, off_partials = 0, off_groups = 0,
+           off_group_tickets = 0, off_ptrs = 0,
            off_tinfo = 0, off_bins_check = 0, off_bins_update = 0, off_segs = 0, off_master = 0,
            off_momentum = 0, off_w16 = 0, total = 0;
 };
@@ -174,6 +177,9 @@ int build_layout(const int64_t* sizes, int32_t n, int32_t check_chunk, int32_t u
     L.off_stats = region(sizeof(StatsBlock));
     L.off_partial_rec = region(sizeof(Partial));
     L.off_partials = region(sizeof(double) * L.bins_check.size());
+    const size_t ngroups = (L.bins_check.size() + kFinishGroup - 1) / kFinishGroup;
+    L.off_groups = region(sizeof(double) * ngroups);
+    L.off_group_tickets = region(sizeof(unsigned int) * ngroups);
     L.off_ptrs = region(sizeof(void*) * (size_t)n);
     L.off_tinfo = region(sizeof(TensorInfo) * (size_t)n);
     L.off_bins_check = region(sizeof(Bin) * L.bins_check.size());
@@ -188,7 +194,25 @@ int build_layout(const int64_t* sizes, int32_t n, int32_t check_chunk, int32_t u
 
 bool finite(float x) { return std::isfinite(x); }
 
-int32_t check_chunk(const mpt_config& c) { return c.check_chunk_elems ? c.check_chunk_elems : kDefaultCheckChunk; }
+// Default check-pass bin: 65536 elements, halved (down to 2048) while the
+// list would give fewer than kMinCheckBins bins (two per SM of a 148-SM
+// B200), so that a small list still spreads over every SM instead of leaving
+// a few CTAs each a long serial loop.  (Many more, shorter bins do not pay:
+// a bin's fixed latency -- table loads, reductions, ticket -- then dominates.)
+constexpr int64_t kMinCheckBins = 296;
+
+int32_t check_chunk(const mpt_config& c, const int64_t* sizes, int32_t n)
+{
+    if (c.check_chunk_elems)
+        return c.check_chunk_elems;
+    int64_t total = 0;
+    for (int32_t i = 0; i < n; ++i)
+        total += sizes[i] > 0 ? sizes[i] : 0;
+    int32_t chunk = kDefaultCheckChunk;
+    while (chunk > kChunkQuantum && total / chunk < kMinCheckBins)
+        chunk /= 2;
+    return chunk;
+}
 int32_t update_chunk(const mpt_config& c) { return c.update_chunk_elems ? c.update_chunk_elems : kDefaultUpdateChunk; }
 
 }  // namespace
@@ -206,6 +230,8 @@ struct mpt_handle {
     StatsBlock* d_stats = nullptr;
     Partial* d_partial_rec = nullptr;     // this rank's record (sharded step)
     double* d_partials = nullptr;
+    double* d_groups = nullptr;
+    unsigned int* d_group_tickets = nullptr;
     const uint16_t** d_ptrs = nullptr;
     TensorInfo* d_tinfo = nullptr;
     Bin* d_bins_check = nullptr;
@@ -226,8 +252,10 @@ struct mpt_handle {
     int32_t clean_run = 0;
     mpt_stats_t stats{};
     bool broken = false;
-    // kernel timing: ring of (start, between, end) events, one per step
-    bool timing = false;
+    // kernel timing: ring of (start, between, end) events, one per timed step;
+    // every timing_every-th step queued since mpt_set_timing is timed
+    int32_t timing_every = 0;
+    int64_t timing_count = 0;
     std::vector<cudaEvent_t> tev;
     int64_t t_head = 0, t_tail = 0;
 };
@@ -314,10 +342,10 @@ static void launch_update_opt(const UpdateArgs& a, bool stale, bool checked, cud
 
 // What the check pass needs from S (the same values the device computes when
 // its state machine sets S): 1/S in binary32 and, for S = 2^e with
-// -15 <= e <= 100, the binary64 constant 2^(1008-e).
+// -15 <= e <= 100, the binary64 constant 2^(-2e) = 1/S^2.
 struct HostScale {
     float inv;
-    double dscale;
+    double sq_unscale;
     int32_t pow2;
 };
 
@@ -328,7 +356,7 @@ static HostScale host_scale_params(float S)
     int e2 = 0;
     const bool pow2 = std::frexp(S, &e2) == 0.5f && (e2 - 1) >= -15 && (e2 - 1) <= 100;
     r.pow2 = pow2 ? 1 : 0;
-    r.dscale = pow2 ? std::ldexp(1.0, 1008 - (e2 - 1)) : 0.0;
+    r.sq_unscale = pow2 ? std::ldexp(1.0, -2 * (e2 - 1)) : 0.0;
     return r;
 }
 
@@ -405,12 +433,14 @@ static int enqueue_step(mpt_handle* h, const void* const* d_grads_half, bool sca
     CheckArgs ca;
     ca.t = t;
     ca.partials = h->d_partials;
+    ca.group_partials = h->d_groups;
+    ca.group_tickets = h->d_group_tickets;
     ca.ctrl = h->d_ctrl;
     ca.host_scale = host_scale;
     {
         const HostScale hp = host_scale_params(scale_on_device ? 1.0f : host_scale);
         ca.host_inv = hp.inv;
-        ca.host_dscale = hp.dscale;
+        ca.host_sq_unscale = hp.sq_unscale;
         ca.host_pow2 = hp.pow2;
     }
     ca.scale_on_device = scale_on_device ? 1 : 0;
@@ -458,7 +488,7 @@ static int enqueue_step(mpt_handle* h, const void* const* d_grads_half, bool sca
     }
 
     cudaEvent_t* ev = nullptr;
-    if (h->timing) {
+    if (h->timing_every > 0 && h->timing_count++ % h->timing_every == 0) {
         if (h->t_head - h->t_tail == kTimingRing && !timing_pop(h))
             return MPT_ERR_CUDA;
         ev = &h->tev[3 * (int)(h->t_head % kTimingRing)];
@@ -540,7 +570,7 @@ static bool upload_scaler_state(mpt_handle* h, float scale, int32_t clean_run)
     return cudaMemcpy(c + offsetof(Ctrl, scale), &scale, sizeof scale, cudaMemcpyHostToDevice) == cudaSuccess &&
            cudaMemcpy(c + offsetof(Ctrl, clean_run), &clean_run, sizeof clean_run, cudaMemcpyHostToDevice) == cudaSuccess &&
            cudaMemcpy(c + offsetof(Ctrl, next_inv), &p.inv, sizeof p.inv, cudaMemcpyHostToDevice) == cudaSuccess &&
-           cudaMemcpy(c + offsetof(Ctrl, next_dscale), &p.dscale, sizeof p.dscale, cudaMemcpyHostToDevice) == cudaSuccess &&
+           cudaMemcpy(c + offsetof(Ctrl, next_sq_unscale), &p.sq_unscale, sizeof p.sq_unscale, cudaMemcpyHostToDevice) == cudaSuccess &&
            cudaMemcpy(c + offsetof(Ctrl, next_pow2), &p.pow2, sizeof p.pow2, cudaMemcpyHostToDevice) == cudaSuccess;
 }
 
@@ -562,7 +592,7 @@ int mpt_workspace_bytes(const int64_t* sizes, int32_t n, const mpt_config* cfg, 
     if (!config_ok(c))
         return MPT_ERR_INVALID_ARG;
     Layout L;
-    const int rc = build_layout(sizes, n, check_chunk(c), update_chunk(c), L);
+    const int rc = build_layout(sizes, n, check_chunk(c, sizes, n), update_chunk(c), L);
     if (rc != MPT_OK)
         return rc;
     *bytes = L.total;
@@ -583,7 +613,7 @@ int mpt_create(const int64_t* sizes, int32_t n, const mpt_config* cfg, void* d_w
         return MPT_ERR_INVALID_ARG;
     h->cfg = c;
     h->n = n;
-    int rc = build_layout(sizes, n, check_chunk(c), update_chunk(c), h->L);
+    int rc = build_layout(sizes, n, check_chunk(c, sizes, n), update_chunk(c), h->L);
     if (rc != MPT_OK) {
         release(h);
         return rc;
@@ -612,6 +642,8 @@ int mpt_create(const int64_t* sizes, int32_t n, const mpt_config* cfg, void* d_w
     h->d_stats = reinterpret_cast<StatsBlock*>(ws + L.off_stats);
     h->d_partial_rec = reinterpret_cast<Partial*>(ws + L.off_partial_rec);
     h->d_partials = reinterpret_cast<double*>(ws + L.off_partials);
+    h->d_groups = reinterpret_cast<double*>(ws + L.off_groups);
+    h->d_group_tickets = reinterpret_cast<unsigned int*>(ws + L.off_group_tickets);
     h->d_ptrs = reinterpret_cast<const uint16_t**>(ws + L.off_ptrs);
     h->d_tinfo = reinterpret_cast<TensorInfo*>(ws + L.off_tinfo);
     h->d_bins_check = reinterpret_cast<Bin*>(ws + L.off_bins_check);
@@ -631,6 +663,7 @@ int mpt_create(const int64_t* sizes, int32_t n, const mpt_config* cfg, void* d_w
               cudaMemcpy(h->d_bins_update, L.bins_update.data(), sizeof(Bin) * L.bins_update.size(), cudaMemcpyHostToDevice) == cudaSuccess &&
               cudaMemcpy(h->d_segs, L.segs.data(), sizeof(Seg) * L.segs.size(), cudaMemcpyHostToDevice) == cudaSuccess &&
               cudaMemset(h->d_ctrl, 0, sizeof(Ctrl)) == cudaSuccess &&
+              cudaMemset(h->d_group_tickets, 0, L.off_ptrs - L.off_group_tickets) == cudaSuccess &&
               cudaMemset(h->d_stats, 0, sizeof(StatsBlock)) == cudaSuccess &&
               cudaMemset(h->d_ptrs, 0, sizeof(void*) * n) == cudaSuccess &&
               cudaMemset(ws + L.off_master, 0, L.total - L.off_master) == cudaSuccess &&
@@ -819,11 +852,11 @@ int mpt_set_scaler_state(mpt_handle* h, float scale, int32_t clean_run)
     return MPT_OK;
 }
 
-int mpt_set_timing(mpt_handle* h, int32_t enable)
+int mpt_set_timing(mpt_handle* h, int32_t every)
 {
-    if (!h)
+    if (!h || every < 0)
         return MPT_ERR_INVALID_ARG;
-    if (enable && h->tev.empty()) {
+    if (every && h->tev.empty()) {
         h->tev.assign(3 * kTimingRing, nullptr);
         for (cudaEvent_t& e : h->tev) {
             if (cudaEventCreate(&e) != cudaSuccess) {
@@ -832,12 +865,13 @@ int mpt_set_timing(mpt_handle* h, int32_t enable)
             }
         }
     }
-    if (!enable) {
+    if (!every) {
         while (h->t_tail < h->t_head)
             if (!timing_pop(h))
                 return fail_cuda(h);
     }
-    h->timing = enable != 0;
+    h->timing_every = every;
+    h->timing_count = 0;
     return MPT_OK;
 }
 
@@ -902,7 +936,7 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratch
 template <bool kPow2>
 __global__ void __launch_bounds__(kThreads)
 check_flat_kernel(const uint16_t* g, int64_t n, unsigned char* scratch, mpt_check_result* out,
-                  float inv_scale, double dscale, float clip)
+                  float inv_scale, double sq_unscale, float clip)
 {
     __shared__ double s_red[kWarps];
     __shared__ unsigned int s_ured[kWarps];
@@ -915,7 +949,7 @@ check_flat_kernel(const uint16_t* g, int64_t n, unsigned char* scratch, mpt_chec
 
     SqParams a{};
     a.inv_scale = inv_scale;
-    a.dscale = dscale;
+    a.sq_unscale = sq_unscale;
     a.pow2 = kPow2;
     SqAcc s;
     check_range<kPow2>(g + begin, len, a, s);
@@ -927,7 +961,7 @@ check_flat_kernel(const uint16_t* g, int64_t n, unsigned char* scratch, mpt_chec
             cnt += ((g[begin + j] & 0x7C00u) == 0x7C00u) ? 1u : 0u;
         nf = block_sum_u32(cnt, s_ured);
     }
-    const double part = block_sum(s.a0 + s.a1, s_red);
+    const double part = unscaled_sum(block_sum(s.a0 + s.a1, s_red), a);
     if (threadIdx.x == 0) {
         partials[blockIdx.x] = part;
         if (nf)
@@ -940,10 +974,7 @@ check_flat_kernel(const uint16_t* g, int64_t n, unsigned char* scratch, mpt_chec
         return;
 
     __threadfence();
-    double x = 0.0;
-    for (int k = threadIdx.x; k < (int)gridDim.x; k += kThreads)
-        x += __ldcg(partials + k);
-    const double sumsq = block_sum(x, s_red);
+    const double sumsq = block_sum(sum_partials(partials, (int)gridDim.x), s_red);
     if (threadIdx.x == 0) {
         const unsigned long long nnf = atomicAdd(&c->nonfinite_acc, 0ull);
         const bool found = nnf != 0;
@@ -1001,13 +1032,13 @@ extern "C" int mpt_check_flat_noalloc(const void* d_grads_half, int64_t n, float
     const float inv_scale = 1.0f / scale;
     int e2 = 0;
     const bool pow2 = std::frexp(scale, &e2) == 0.5f && (e2 - 1) >= -15 && (e2 - 1) <= 100;
-    const double dscale = pow2 ? std::ldexp(1.0, 1008 - (e2 - 1)) : 0.0;
+    const double sq_unscale = pow2 ? std::ldexp(1.0, -2 * (e2 - 1)) : 0.0;
     const unsigned int bins = (unsigned int)((n + kNoAllocChunk - 1) / kNoAllocChunk);
     const uint16_t* g = static_cast<const uint16_t*>(d_grads_half);
     if (pow2)
-        check_flat_kernel<true><<<bins, kThreads, 0, st>>>(g, n, scratch, d_result, inv_scale, dscale, clip);
+        check_flat_kernel<true><<<bins, kThreads, 0, st>>>(g, n, scratch, d_result, inv_scale, sq_unscale, clip);
     else
-        check_flat_kernel<false><<<bins, kThreads, 0, st>>>(g, n, scratch, d_result, inv_scale, dscale, clip);
+        check_flat_kernel<false><<<bins, kThreads, 0, st>>>(g, n, scratch, d_result, inv_scale, sq_unscale, clip);
     if (cudaGetLastError() != cudaSuccess)
         return MPT_ERR_CUDA;
     return MPT_OK;

@@ -16,6 +16,8 @@ constexpr int kMaxChunk = 1 << 20;
 constexpr int kSmallTensor = 1024;         // tensors up to this size are packed
 constexpr int kPackedMaxElems = 4096;      // elements per packed bin
 constexpr int kMaxPackedSegs = 256;        // tensors per packed bin
+constexpr int kFinishGroup = 64;           // check bins per first-level finish group
+static_assert(kFinishGroup <= kThreads, "one thread per bin of a finish group");
 constexpr int kPackedUnroll = kPackedMaxElems / kThreads;  // elements per thread
 
 enum BinKind : int32_t {
@@ -53,17 +55,24 @@ struct __align__(16) TensorInfo {
 
 // Device control block.  The check kernel accumulates into the *_acc fields,
 // and its last CTA turns them into the step result, then clears every
-// accumulator (its own and the update kernel's) for the next step.
-struct __align__(16) Ctrl {
-    // check-kernel accumulators
+// accumulator (its own and the update kernel's) for the next step.  The two
+// kernels' atomic accumulators and the fields that every CTA reads when it
+// starts (S, 1/S, the skip flag, the clip coefficient) sit on three separate
+// 128-byte lines, so that a CTA's first read never queues behind the other
+// CTAs' atomics on the same line.
+struct __align__(128) Ctrl {
+    // line 0: check-kernel accumulators
     unsigned long long nonfinite_acc;
     unsigned int ticket;
     unsigned int error_acc;
-    // update-kernel accumulators (cleared by the check kernel's last CTA)
+    unsigned int max_mag_acc;  // statistics mode: largest finite |g16| (atomicMax)
+    unsigned int pad0[27];
+    // line 1: update-kernel accumulators (cleared by the check kernel's last CTA)
     unsigned long long zero_acc;
     unsigned long long subnormal_acc;
     unsigned long long stale_acc;
-    // step result written by the check kernel's last CTA
+    unsigned int pad1[26];
+    // line 2: step result written by the check kernel's last CTA
     double sumsq;
     double norm;
     unsigned long long n_nonfinite;
@@ -78,16 +87,17 @@ struct __align__(16) Ctrl {
     int32_t clean_run;     // consecutive clean steps so far
     unsigned long long steps_total;
     unsigned long long skipped_total;
-    // gradient statistics (statistics mode): largest finite |g16| pattern
-    unsigned int max_mag_acc;  // accumulated by the check CTAs (atomicMax)
-    unsigned int max_mag;      // the last step's
-    float max_abs;             // its unscaled value, fp32(max|g16|) * (1/S)
+    // gradient statistics (statistics mode): the last step's largest finite
+    // |g16| pattern and its unscaled value, fp32(max|g16|) * (1/S)
+    unsigned int max_mag;
+    float max_abs;
     // what the next check pass needs from `scale`, computed once when the
-    // state is set (1/S and, for S = 2^e with -15 <= e <= 100, 2^(1008-e))
+    // state is set (1/S and, for S = 2^e with -15 <= e <= 100, 2^(-2e))
     int32_t next_pow2;
-    double next_dscale;
+    unsigned int pad2;
+    double next_sq_unscale;
     float next_inv;
-    unsigned int pad;
+    unsigned int pad3;
 };
 
 // What one rank's check pass contributes to a sharded step (32 bytes): its

@@ -50,10 +50,12 @@ struct ScalerParams {
 struct CheckArgs {
     Tables t;
     double* partials;     // one binary64 partial sum of squares per bin
+    double* group_partials;        // one per group of kFinishGroup bins
+    unsigned int* group_tickets;   // one per group; zero between launches
     Ctrl* ctrl;
     float host_scale;     // S the gradients carry, when given by the host,
     float host_inv;       // with its binary32 reciprocal
-    double host_dscale;   // and 2^(1008-e) when S = 2^e, -15 <= e <= 100
+    double host_sq_unscale;  // and 2^(-2e) when S = 2^e, -15 <= e <= 100
     int32_t host_pow2;
     int32_t scale_on_device;  // 1: S is ctrl->scale (asynchronous steps)
     float clip;           // <= 0: off
@@ -76,10 +78,12 @@ struct UpdateArgs {
 };
 
 // What the squares need from S: the binary32 reciprocal 1/S and, when S is a
-// power of two 2^e with -15 <= e <= 100, the binary64 constant 2^(1008-e).
+// power of two 2^e with -15 <= e <= 100, the binary64 constant 2^(-2e) that
+// turns a sum of squared scaled gradients into the sum of squared unscaled
+// ones.
 struct SqParams {
     float inv_scale;
-    double dscale;
+    double sq_unscale;
     bool pow2;
 };
 
@@ -91,7 +95,7 @@ __device__ __forceinline__ SqParams sq_params(float S)
     const int biased = (int)((b >> 23) & 0xFFu);
     const int e = biased - 127;
     q.pow2 = (b & 0x807FFFFFu) == 0 && biased != 0 && e >= -15 && e <= 100;
-    q.dscale = q.pow2 ? __longlong_as_double((long long)(1008 - e + 1023) << 52) : 0.0;
+    q.sq_unscale = q.pow2 ? __longlong_as_double((long long)(1023 - 2 * e) << 52) : 0.0;
     return q;
 }
 
@@ -147,7 +151,7 @@ __device__ __forceinline__ void finish_step(Ctrl* c, float S, const SqParams& q,
     c->scale = next;
     const SqParams nq = sq_params(next);
     c->next_inv = nq.inv_scale;
-    c->next_dscale = nq.dscale;
+    c->next_sq_unscale = nq.sq_unscale;
     c->next_pow2 = nq.pow2 ? 1 : 0;
     c->clean_run = clean;
     c->steps_total += 1;
@@ -220,53 +224,59 @@ __device__ __forceinline__ uint32_t h2_bits(__half2 h)
 
 struct SqAcc {
     double a0 = 0.0, a1 = 0.0;
-    uint32_t nf = 0;  // bit 15 or 31 set <=> some element seen was +-inf/NaN
 
-    __device__ __forceinline__ bool saw_nonfinite() const { return (nf & 0x80008000u) != 0; }
+    // Some element this thread saw was +-inf/NaN: the square of an inf or a
+    // NaN is inf or NaN and stays so through every later addition, while a
+    // sum of finite squares cannot overflow binary64 (each square is at most
+    // 65504^2 / min(S, 1)^2).  With S not a power of two a huge 1/S can make
+    // the binary32 product of a finite gradient inf; that only sends the CTA
+    // through its exact recount, which then finds no non-finite element.
+    __device__ __forceinline__ bool saw_nonfinite() const { return !isfinite(a0 + a1); }
 };
 
-// Square of one unscaled gradient, accumulated in binary64.
+// Square of one gradient, accumulated in binary64.
 //
-// Power-of-two S: x = fp32(g16) * (1/S) is exact, so x can be formed in
-// binary64 straight from the binary16 bits.  The 15 magnitude bits are placed
-// in the high word of a binary64 so that its exponent field is the binary16
-// exponent field and its top fraction bits are the binary16 fraction; that
-// number is the binary16 value times 2^-1008 (binary16 subnormals become
-// binary64 subnormals with the same scale), and one multiply by 2^1008 / S
-// gives x exactly.  The square of an 11-bit significand is exact, so the FMA
-// rounds once, like the sum x*x + acc of the definition.
+// Power-of-two S: x = fp32(g16) * (1/S) is exact, and so is the product of a
+// binary64 sum with a power of two that stays in range.  So the squares of
+// the scaled gradients themselves are summed -- widened exactly to binary64
+// by the hardware conversions, squared exactly (an 11-bit significand) and
+// added with one rounding each, like x*x + acc of the definition -- and the
+// CTA's total is multiplied once by 2^(-2e) = 1/S^2 (SqParams::sq_unscale).
+// Every partial sum is then the definition's partial sum times S^2, exactly,
+// so the result is bit for bit that of summing x*x.
 //
 // Other S: x is rounded to binary32 first, as the definition says.
 template <bool kPow2>
-__device__ __forceinline__ void sq_bits(uint32_t mag_hi_word, uint16_t h, const SqParams& a,
-                                        double& acc)
+__device__ __forceinline__ double sq_value(float g, const SqParams& a)
 {
-    if constexpr (kPow2) {
-        const double x = __hiloint2double((int)mag_hi_word, 0) * a.dscale;
-        acc = fma(x, x, acc);
-    } else {
-        const double x = (double)__fmul_rn(__half2float(__ushort_as_half(h)), a.inv_scale);
-        acc = fma(x, x, acc);
-    }
+    if constexpr (kPow2)
+        return (double)g;
+    else
+        return (double)__fmul_rn(g, a.inv_scale);
 }
 
 template <bool kPow2>
 __device__ __forceinline__ void sq_word(uint32_t w, const SqParams& a, SqAcc& s)
 {
-    sq_bits<kPow2>((w << 10) & 0x01FFFC00u, (uint16_t)(w & 0xFFFFu), a, s.a0);
-    sq_bits<kPow2>((w >> 6) & 0x01FFFC00u, (uint16_t)(w >> 16), a, s.a1);
-    // Lane is +-inf/NaN <=> its exponent bits are all ones <=> (~w & 0x7C00)
-    // is 0 in that lane; subtracting 0x0400 per lane then borrows into bit 15
-    // (bit 31).  A borrow out of the low lane only reaches the high lane when
-    // the low lane is itself non-finite, so the flag is exact.
-    s.nf |= (~w & 0x7C007C00u) - 0x04000400u;
+    const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&w));
+    const double x0 = sq_value<kPow2>(f.x, a);
+    const double x1 = sq_value<kPow2>(f.y, a);
+    s.a0 = fma(x0, x0, s.a0);
+    s.a1 = fma(x1, x1, s.a1);
 }
 
 template <bool kPow2>
 __device__ __forceinline__ void sq_half(uint16_t h, const SqParams& a, SqAcc& s)
 {
-    sq_bits<kPow2>(((uint32_t)h << 10) & 0x01FFFC00u, h, a, s.a0);
-    s.nf |= (~(uint32_t)h & 0x7C00u) - 0x0400u;
+    const double x = sq_value<kPow2>(__half2float(__ushort_as_half(h)), a);
+    s.a0 = fma(x, x, s.a0);
+}
+
+// A CTA's sum of squares in the definition's scale (power-of-two S: the sum
+// of the scaled squares times 1/S^2, exact).
+__device__ __forceinline__ double unscaled_sum(double part, const SqParams& a)
+{
+    return a.pow2 ? part * a.sq_unscale : part;
 }
 
 template <bool kPow2>
@@ -421,6 +431,28 @@ __device__ __forceinline__ double block_sum(double x, double* red)
     return t;
 }
 
+// This thread's share of the per-bin partials, k = threadIdx.x + i*kThreads in
+// increasing i, with eight loads issued before they are added (the same order
+// of additions as one load at a time).
+__device__ __forceinline__ double sum_partials(const double* partials, int n)
+{
+    constexpr int kU = 8;
+    double x = 0.0;
+    int k = threadIdx.x;
+    for (; k + (kU - 1) * kThreads < n; k += kU * kThreads) {
+        double p[kU];
+#pragma unroll
+        for (int i = 0; i < kU; ++i)
+            p[i] = __ldcg(partials + k + i * kThreads);
+#pragma unroll
+        for (int i = 0; i < kU; ++i)
+            x += p[i];
+    }
+    for (; k < n; k += kThreads)
+        x += __ldcg(partials + k);
+    return x;
+}
+
 __device__ __forceinline__ unsigned int block_sum_u32(unsigned int x, unsigned int* red)
 {
     x = __reduce_add_sync(0xffffffffu, x);
@@ -525,12 +557,12 @@ __global__ void __launch_bounds__(kThreads, kStats == kMaxHist ? 4 : 8) check_ke
         const Ctrl* c = a.ctrl;
         S = c->scale;
         q.inv_scale = c->next_inv;
-        q.dscale = c->next_dscale;
+        q.sq_unscale = c->next_sq_unscale;
         q.pow2 = c->next_pow2 != 0;
     } else {
         S = a.host_scale;
         q.inv_scale = a.host_inv;
-        q.dscale = a.host_dscale;
+        q.sq_unscale = a.host_sq_unscale;
         q.pow2 = a.host_pow2 != 0;
     }
     SqAcc s;
@@ -611,7 +643,7 @@ __global__ void __launch_bounds__(kThreads, kStats == kMaxHist ? 4 : 8) check_ke
         nf = block_sum_u32(c, s_ured);
     }
 
-    const double part = block_sum(s.a0 + s.a1, s_red);
+    const double part = unscaled_sum(block_sum(s.a0 + s.a1, s_red), q);
     if constexpr (kStats != kNoStats) {
         const unsigned int mx = block_max_u32(sa.mx, s_ured);   // ends with __syncthreads
         if (kStats == kMaxHist && threadIdx.x < 32) {
@@ -632,23 +664,40 @@ __global__ void __launch_bounds__(kThreads, kStats == kMaxHist ? 4 : 8) check_ke
         if (!valid)
             atomicOr(&a.ctrl->error_acc, (unsigned int)kErrBadBin);
     }
+    // Two-level finish, so that the serial work after the last bin is small:
+    // the last CTA to complete in each group of kFinishGroup consecutive bins
+    // adds that group's partials (in bin order, fixed pattern); the last
+    // group to complete adds the group sums (in group order) and finishes the
+    // step.  Fences before each ticket make every counter and partial written
+    // before it visible to the CTA that draws the last ticket.
     __syncthreads();  // every write of this CTA precedes its ticket
+    const int grp = (int)blockIdx.x / kFinishGroup;
+    const int g_begin = grp * kFinishGroup;
+    const int g_len = min(kFinishGroup, (int)gridDim.x - g_begin);
     if (threadIdx.x == 0) {
         __threadfence();
-        const unsigned int ticket = atomicAdd(&a.ctrl->ticket, 1u);
-        s_last = (ticket == gridDim.x - 1);
+        s_last = atomicAdd(&a.group_tickets[grp], 1u) == (unsigned int)g_len - 1;
+    }
+    __syncthreads();
+    if (!s_last)
+        return;
+    __threadfence();
+    const double gsum = block_sum(
+        threadIdx.x < g_len ? __ldcg(a.partials + g_begin + threadIdx.x) : 0.0, s_red);
+    const int ngroups = ((int)gridDim.x + kFinishGroup - 1) / kFinishGroup;
+    if (threadIdx.x == 0) {
+        a.group_partials[grp] = gsum;
+        a.group_tickets[grp] = 0;
+        __threadfence();
+        s_last = atomicAdd(&a.ctrl->ticket, 1u) == (unsigned int)ngroups - 1;
     }
     __syncthreads();
     if (!s_last)
         return;
 
-    // Last CTA: every other CTA's partial and counters are visible.  Sum the
-    // partials in bin order with a fixed pattern, then write the result.
+    // Last group: every CTA's partial and counters are visible.
     __threadfence();
-    double x = 0.0;
-    for (int k = threadIdx.x; k < t.nbins; k += kThreads)
-        x += __ldcg(a.partials + k);
-    const double sumsq = block_sum(x, s_red);
+    const double sumsq = block_sum(sum_partials(a.group_partials, ngroups), s_red);
     Ctrl* c = a.ctrl;
     if constexpr (kStats == kMaxHist) {
         if (threadIdx.x < 32) {
@@ -703,7 +752,7 @@ __global__ void finish_kernel(FinishArgs a)
     Ctrl* c = a.ctrl;
     SqParams q;
     q.inv_scale = c->next_inv;
-    q.dscale = c->next_dscale;
+    q.sq_unscale = c->next_sq_unscale;
     q.pow2 = c->next_pow2 != 0;
     finish_step(c, c->scale, q, nf, sumsq, mm, a.have_max != 0, err, a.clip, a.scaler);
 }

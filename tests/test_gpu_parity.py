@@ -210,6 +210,14 @@ def test_stats_and_timing():
     assert st["steps"] == 3 and st["timed_steps"] == 3
     assert st["check_ms_total"] > 0 and st["update_ms_total"] > 0
     assert st["scale"] == p.scale
+    # sampled: every third step from the next one on
+    p.opt.set_timing(3)
+    for _ in range(7):
+        p.step()
+    assert p.opt.stats()["timed_steps"] == 3 + 3
+    p.opt.set_timing(0)
+    p.step()
+    assert p.opt.stats()["timed_steps"] == 6
 
 
 # ---------------------------------------------------------------------------
