@@ -46,6 +46,9 @@ DEFAULT_WORKLOAD = "gpt2_medium"
 BYTES_UPDATE = 20        # per parameter: read g16 2 + w 4 + v 4, write w 4 + v 4 + w16 2
 BYTES_CHECK = 2          # per parameter: read g16
 TIMING_EVERY = 10       # kernel events on every 10th timed step
+SKIP_STEPS = 20         # overflow steps timed apart
+BYTES_SKIP = 4          # per parameter on an overflow step: check 2 + counting pass 2
+NOMINAL_HBM_GBS = 8000.0
 L2_BYTES = 126 * 2 ** 20
 READBACK_BYTES = 384     # the control block mpt_step copies back each step
 FALLBACK_HBM_GBS = 6650.0
@@ -311,6 +314,35 @@ def run_mpt(args, cfg):
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         ms_max = float(t.item())
 
+    # overflow (skipped) steps, reported apart: one +inf planted in the
+    # gradients, so every step takes the skip path -- the check pass plus the
+    # update kernel's counting pass (4 B/param) -- and halves S on the device
+    skip_steps = SKIP_STEPS
+    flat0 = sets[0]
+    saved = flat0[0].item()
+    flat0[0] = 0x7C00
+    for k in range(2):
+        step(0)
+    opt.wait(stream)
+    s_before = opt.stats()["skipped"]
+    barrier()
+    torch.cuda.synchronize(dev)
+    g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    g0.record(stream)
+    for k in range(skip_steps):
+        step(0)
+    g1.record(stream)
+    opt.wait(stream)
+    torch.cuda.synchronize(dev)
+    skip_ms = g0.elapsed_time(g1) / skip_steps
+    skip_all = opt.stats()["skipped"] - s_before == skip_steps
+    flat0[0] = saved
+    opt.set_scaler_state(S, 0)
+    if world > 1:
+        t = torch.tensor([skip_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        skip_ms = float(t.item())
+
     # end to end through the public API: gradients from pinned host memory
     # every step, result read back by the call itself
     host = [torch.empty(g.numel(), dtype=torch.int16, pin_memory=True) for g in sets]
@@ -356,6 +388,7 @@ def run_mpt(args, cfg):
             "data": "synthetic (seeded FP16 gradients, random-init FP32 masters)",
             "hbm_gbs": (BYTES_UPDATE + BYTES_CHECK) * P / (ms_step * 1e-3) / 1e9,
             "hbm_frac_of_measured": (BYTES_UPDATE + BYTES_CHECK) * P / (ms_step * 1e-3) / 1e9 / peak,
+            "hbm_frac_of_nominal_8tbs": (BYTES_UPDATE + BYTES_CHECK) * P / (ms_step * 1e-3) / 1e9 / NOMINAL_HBM_GBS,
             "config": {"workload": cfg.name, "params": P, "tensors": len(cfg.sizes),
                        "bytes_per_param": BYTES_UPDATE + BYTES_CHECK,
                        "scale": S, "clip": cfg.clip, "lr": cfg.lr, "momentum": cfg.momentum,
@@ -372,11 +405,15 @@ def run_mpt(args, cfg):
             "roofline": {"kernel": "update_kernel", "bound": "hbm",
                          "achieved": achieved_update, "peak": peak, "unit": "GB/s",
                          "frac": achieved_update / peak, "peak_kind": peak_kind,
+                         "frac_of_nominal_8tbs": achieved_update / NOMINAL_HBM_GBS,
                          "traffic": traffic,
                          "algorithmic_bytes_per_launch": BYTES_UPDATE * P,
                          "check_kernel": {"achieved": achieved_check,
                                           "frac": achieved_check / peak,
                                           "algorithmic_bytes_per_launch": BYTES_CHECK * P}},
+            "skipped_step": {"ms": skip_ms, "steps": skip_steps, "all_skipped": skip_all,
+                             "bytes_per_param": BYTES_SKIP,
+                             "gbs": BYTES_SKIP * P / (skip_ms * 1e-3) / 1e9},
             "e2e": {"value": world * P / (e2e_ms * 1e-3), "unit": "params/s",
                     "ms_per_step": e2e_ms,
                     "h2d_bytes_per_step": sets[0].numel() * 2,

@@ -467,6 +467,8 @@ static int enqueue_step(mpt_handle* h, const void* const* d_grads_half, bool sca
     ua.mu = momentum;
     ua.wd = weight_decay;
     ua.eps = h->cfg.eps;
+    ua.check_bins = h->d_bins_check;
+    ua.check_nbins = (int32_t)h->L.bins_check.size();
 
     const bool checked = (h->cfg.flags & MPT_FLAG_CHECKED) != 0;
     const bool stale = (h->cfg.flags & MPT_FLAG_COUNT_STALE) != 0;

@@ -3,9 +3,10 @@
 //   check_kernel   one pass over the FP16 gradients: overflow check (Step 6 of
 //                  "The Integrated Training Procedure (Figure 1)"), sum of
 //                  squares of the unscaled gradients (global-L2 clip), with a
-//                  deterministic last-CTA finish that writes the step result
+//                  deterministic two-level finish that writes the step result
 //   update_kernel  the fused per-element update (Steps 5 and 7, weight decay,
-//                  clip, FP16 copy); on an overflow step it only counts
+//                  clip, FP16 copy); on an overflow step its first CTAs only
+//                  count zero and subnormal gradients, the rest exit
 //   refresh_kernel FP16 copy = round-to-nearest-even(master) (Step 1)
 //
 // All three are HBM-bound streaming kernels on the CUDA cores: there is no
@@ -75,6 +76,8 @@ struct UpdateArgs {
     float mu;
     float wd;
     float eps;            // Adagrad only
+    const Bin* check_bins;  // the check pass's (larger) bins: the counting
+    int32_t check_nbins;    // sweep of an overflow step walks these
 };
 
 // What the squares need from S: the binary32 reciprocal 1/S and, when S is a
@@ -918,13 +921,30 @@ __device__ __forceinline__ void update_range(const uint16_t* g, float* w, float*
 }
 
 // Overflow step: the update is skipped; only the range counts are taken.
+// Zero / subnormal counts of one contiguous range (16-B loads, four in
+// flight per thread, when the range is 16-B aligned).
 __device__ __forceinline__ void count_range(const uint16_t* g, int len, uint32_t& nz2, uint32_t& ns2)
 {
     int start = 0;
     if ((reinterpret_cast<uintptr_t>(g) & 15) == 0) {
+        constexpr int kU = 4;
         const uint4* gv = reinterpret_cast<const uint4*>(g);
         const int nv = len >> 3;
-        for (int i = threadIdx.x; i < nv; i += kThreads) {
+        int i = threadIdx.x;
+        for (; i + (kU - 1) * kThreads < nv; i += kU * kThreads) {
+            uint4 q[kU];
+#pragma unroll
+            for (int k = 0; k < kU; ++k)
+                q[k] = __ldcs(gv + i + k * kThreads);
+#pragma unroll
+            for (int k = 0; k < kU; ++k) {
+                count_word(q[k].x, nz2, ns2);
+                count_word(q[k].y, nz2, ns2);
+                count_word(q[k].z, nz2, ns2);
+                count_word(q[k].w, nz2, ns2);
+            }
+        }
+        for (; i < nv; i += kThreads) {
             const uint4 q = __ldcs(gv + i);
             count_word(q.x, nz2, ns2);
             count_word(q.y, nz2, ns2);
@@ -937,8 +957,55 @@ __device__ __forceinline__ void count_range(const uint16_t* g, int len, uint32_t
         count_half(__ldcs(g + j), nz2, ns2);
 }
 
+// CTAs of an overflow step's update grid that take the range counts; the
+// rest exit at once.  592 = 4 CTAs (the update kernel's residency) per SM.
+constexpr int kCountCtas = 592;
+
+// Overflow step: nothing is updated, and the zero and subnormal counts are
+// taken by a sweep of the check pass's bins (64K-element ranges and the
+// packed bins): CTA k counts bins k, k + sweepers, ...  A bin's lane-packed
+// counts stay below 2^12 per lane (at most 2^20 elements per bin).
+template <bool kChecked>
+__device__ __forceinline__ void count_sweep(const Tables& t, const Bin* bins, int nbins,
+                                            int sweepers, Ctrl* ctrl, PackedStage& st,
+                                            unsigned int* s_ured)
+{
+    // t: segments, tensors and pointers (shared by both bin tables)
+    unsigned int n_el = 0, nz = 0, ns = 0;
+    bool bad = false;
+    for (int b = (int)blockIdx.x; b < nbins; b += sweepers) {
+        const Bin bin = bins[b];
+        if (kChecked && !bin_ok(bin, t)) {
+            bad = true;
+            continue;
+        }
+        uint32_t nz2 = 0, ns2 = 0;
+        if (bin.kind == kChunkBin) {
+            count_range(t.grads[bin.tensor] + bin.tensor_begin, bin.n_elems, nz2, ns2);
+        } else {
+            __syncthreads();  // nobody still reads the previous staging
+            stage_packed(bin, t, st);
+            for (int j = threadIdx.x; j < bin.n_elems; j += kThreads) {
+                const int k = find_seg(st.begin, bin.n_segs, j);
+                count_half(__ldcs(st.gptr[k] + (j - st.begin[k])), nz2, ns2);
+            }
+        }
+        nz += (nz2 & 0xFFFFu) + (nz2 >> 16);
+        ns += (ns2 & 0xFFFFu) + (ns2 >> 16);
+        n_el += (unsigned int)bin.n_elems;
+    }
+    const unsigned int bnz = block_sum_u32(nz, s_ured);
+    const unsigned int bns = block_sum_u32(ns, s_ured);
+    if (threadIdx.x == 0) {
+        atomicAdd(&ctrl->zero_acc, (unsigned long long)(n_el - bnz));
+        atomicAdd(&ctrl->subnormal_acc, (unsigned long long)(bnz - bns));
+        if (bad)
+            atomicOr(&ctrl->error, (unsigned int)kErrBadBin);
+    }
+}
+
 template <int kOpt, bool kStale, bool kChecked>
-__global__ void __launch_bounds__(kThreads) update_kernel(UpdateArgs a)
+__global__ void __launch_bounds__(kThreads, kOpt == kOptAdagrad ? 3 : 4) update_kernel(UpdateArgs a)
 {
     __shared__ PackedStage st;
     __shared__ unsigned int s_ured[kWarps];
@@ -954,8 +1021,13 @@ __global__ void __launch_bounds__(kThreads) update_kernel(UpdateArgs a)
 
     // While the check kernel drains, start this CTA's first reads: a bulk
     // (TMA) prefetch of the start of its master, momentum and gradient ranges
-    // into L2.  They do not depend on the check result.
-    if (valid && bin.kind == kChunkBin && threadIdx.x == 0) {
+    // into L2.  Whether to prefetch follows the overflow flag as the check
+    // kernel left it, read alongside the bin: this step's flag for a CTA that
+    // starts after the check has finished (most of the grid), the previous
+    // step's for one that starts while it drains.  It is only a hint: the
+    // update itself reads the flag after the wait.
+    if (valid && bin.kind == kChunkBin && threadIdx.x == 0 &&
+        *reinterpret_cast<const volatile int32_t*>(&a.ctrl->found_inf) == 0) {
         const int n_pre = min(bin.n_elems, kPrefetchElems) & ~7;
         if (n_pre > 0) {
             prefetch_l2(a.master + bin.arena_begin, (uint32_t)n_pre * 4u);
@@ -969,18 +1041,25 @@ __global__ void __launch_bounds__(kThreads) update_kernel(UpdateArgs a)
     // (returns at once when this grid was launched without overlap).
     asm volatile("griddepcontrol.wait;" ::: "memory");
     const Ctrl* c = a.ctrl;
-    const bool skip = c->found_inf != 0;
+    if (c->found_inf != 0) {
+        // Overflow step (Step 6): master, momentum and FP16 copy stay as they
+        // are.  The flag is the same for every thread of the grid, so the
+        // branch is uniform.  (Checked mode: the sweep validates the check
+        // bins it walks; this grid's own bins are validated on the next step
+        // that uses them.)
+        const int sweepers = min(kCountCtas, (int)gridDim.x);
+        if ((int)blockIdx.x < sweepers)
+            count_sweep<kChecked>(t, a.check_bins, a.check_nbins, sweepers, a.ctrl, st, s_ured);
+        return;
+    }
     const UpdParams p{c->inv_scale, c->coef, a.lr, a.mu, a.wd, a.eps};
     uint32_t nz2 = 0, ns2 = 0, stale = 0;
 
     if (valid) {
         if (bin.kind == kChunkBin) {
             const uint16_t* g = t.grads[bin.tensor] + bin.tensor_begin;
-            if (skip)
-                count_range(g, bin.n_elems, nz2, ns2);
-            else
-                update_range<kOpt, kStale>(g, a.master + bin.arena_begin, a.momentum + bin.arena_begin,
-                                     a.w16 + bin.arena_begin, bin.n_elems, p, nz2, ns2, stale);
+            update_range<kOpt, kStale>(g, a.master + bin.arena_begin, a.momentum + bin.arena_begin,
+                                       a.w16 + bin.arena_begin, bin.n_elems, p, nz2, ns2, stale);
         } else {
             stage_packed(bin, t, st);
             constexpr int kU = 4;
@@ -997,10 +1076,8 @@ __global__ void __launch_bounds__(kThreads) update_kernel(UpdateArgs a)
                         const int off = j - st.begin[k];
                         gh[i] = __ldcs(st.gptr[k] + off);
                         e[i] = st.arena[k] + off;
-                        if (!skip) {
-                            w[i] = __ldcs(a.master + e[i]);
-                            v[i] = __ldcs(a.momentum + e[i]);
-                        }
+                        w[i] = __ldcs(a.master + e[i]);
+                        v[i] = __ldcs(a.momentum + e[i]);
                     }
                 }
 #pragma unroll
@@ -1008,14 +1085,12 @@ __global__ void __launch_bounds__(kThreads) update_kernel(UpdateArgs a)
                     if (e[i] < 0)
                         continue;
                     count_half(gh[i], nz2, ns2);
-                    if (!skip) {
-                        const float w0 = w[i];
-                        upd1<kOpt>(__half2float(__ushort_as_half(gh[i])), w[i], v[i], p);
-                        __stcs(a.master + e[i], w[i]);
-                        __stcs(a.momentum + e[i], v[i]);
-                        a.w16[e[i]] = __half_as_ushort(__float2half_rn(w[i]));
-                        stale1<kStale>(w0, w[i], stale);
-                    }
+                    const float w0 = w[i];
+                    upd1<kOpt>(__half2float(__ushort_as_half(gh[i])), w[i], v[i], p);
+                    __stcs(a.master + e[i], w[i]);
+                    __stcs(a.momentum + e[i], v[i]);
+                    a.w16[e[i]] = __half_as_ushort(__float2half_rn(w[i]));
+                    stale1<kStale>(w0, w[i], stale);
                 }
             }
         }

@@ -121,6 +121,44 @@ def test_non_power_of_two_and_extreme_scales(scale):
     p.step()
 
 
+@pytest.mark.parametrize("scale,law", [
+    (2.0 ** -15, (-9.0, 30.0)),     # lowest exponent of the exact power-of-two path
+    (2.0 ** -16, (-8.0, 31.0)),     # just below it: binary32 products first
+    (2.0 ** 100, (-124.0, -85.0)),  # highest exponent of the power-of-two path
+    (2.0 ** 101, (-125.0, -86.0)),  # just above it
+    (2.0 ** 127, (-151.0, -112.0)), # 1/S subnormal: products round in the subnormal range
+])
+def test_scale_exponent_edges(scale, law):
+    """S = 2^e at and beyond the ends of the range where the check pass sums
+    the squares of the scaled gradients and multiplies by 2^(-2e) once; the
+    gradients are drawn so that |g S| spans the binary16 range."""
+    cfg = custom([50_000, 999, 70_001], law=("log2_uniform",) + law, scale0=scale, steps=2)
+    p = Pair(cfg)
+    p.step()
+    p.step()
+
+
+def test_huge_inverse_scale_overflows_products_not_the_check():
+    """S = 2^-120: the binary32 products fp32(g16) * (1/S) of the larger
+    gradients overflow to inf although every gradient is finite.  The
+    definition then has an infinite sum of squares, but no non-finite
+    gradient: the step is not skipped, and the state (with its infinities,
+    no NaN after one step from zero momentum) matches the oracle bit for bit."""
+    cfg = custom([70_000, 3001], law=("log2_uniform", 112.0, 130.0), scale0=2.0 ** -120, steps=1)
+    p = Pair(cfg)
+    host = p.grads(1, p.scale)
+    p.flat.copy_(host)
+    hv = [v.numpy().view(np.uint16) for v in p.layout.views(host)]
+    r = p.opt.step(p.gviews, p.scale, cfg.lr, cfg.momentum, cfg.weight_decay, 0.0)
+    ro = oracle.step(p.state, hv, p.scale, cfg.lr, cfg.momentum, cfg.weight_decay, clip=0.0,
+                     cfg=p.ocfg)
+    assert ro["found_inf"] == 0 and r["found_inf"] == 0 and r["n_nonfinite"] == 0
+    assert math.isinf(ro["norm"]) and math.isinf(r["grad_norm"]) and r["clip_coef"] == 1.0
+    assert r["n_zero"] == ro["n_zero"] and r["n_subnormal"] == ro["n_subnormal"]
+    assert r["new_scale"] == ro["new_scale"]
+    p.compare_state("huge 1/S", exact=True)
+
+
 def test_checked_mode_and_stale_counts():
     cfg = custom([100_000, 17, 3000], steps=3, lr=1e-3)
     p = Pair(cfg, flags=MPT_FLAG_CHECKED | MPT_FLAG_COUNT_STALE)
