@@ -208,8 +208,16 @@ int mpt_step(mpt_handle* h, const void* const* d_grads_half, float scale,
  * from a loss multiplied by that device value, and the step advances the
  * state on the device.  Nothing is read back; call mpt_wait for the result
  * of the last queued step.  The gradient buffers must stay unchanged until
- * the queued work has run.  Errors: MPT_ERR_INVALID_ARG, MPT_ERR_CUDA,
- * MPT_ERR_BROKEN. */
+ * the queued work has run.
+ * CUDA graphs: when d_grads_half holds the same pointers as the previous
+ * step of this handle, the call queues exactly the two kernel launches (no
+ * copy, no host synchronisation), so it can be captured into a CUDA graph
+ * (kernel timing off).  Each replay reads the gradients its buffers hold at
+ * replay time and reads and advances the device scale state; mpt_wait on
+ * the replay stream returns the replayed step's result.  With new pointers
+ * the call first copies the pointer table from pinned host memory, which a
+ * capture must not record.
+ * Errors: MPT_ERR_INVALID_ARG, MPT_ERR_CUDA, MPT_ERR_BROKEN. */
 int mpt_step_async(mpt_handle* h, const void* const* d_grads_half, float lr,
                    float momentum, float weight_decay, float clip, void* cuda_stream);
 

@@ -93,12 +93,17 @@ class Sampled:
             total.sumsq += r.sumsq
         return total
 
-    def step(self, k):
+    def step(self, k, queued=False):
         cfg = self.cfg
         W.make_grads(cfg, k, self.scale, self.layout, "cuda", out=self.flat)
         self.host.copy_(self.flat)
-        r = self.opt.step(self.views, self.scale, cfg.lr, cfg.momentum, cfg.weight_decay,
-                          cfg.clip)
+        if queued:
+            # the benchmark's path: S is the device state the previous step left
+            self.opt.step_async(self.views, cfg.lr, cfg.momentum, cfg.weight_decay, cfg.clip)
+            r = self.opt.wait()
+        else:
+            r = self.opt.step(self.views, self.scale, cfg.lr, cfg.momentum, cfg.weight_decay,
+                              cfg.clip)
         ro = oracle.clip_coef(self.full_check(self.scale), cfg.clip)
         for key in ("found_inf", "clipped", "n_zero", "n_subnormal", "n_nonfinite"):
             assert r[key] == getattr(ro, key), (k, key, r[key], getattr(ro, key))
@@ -125,10 +130,10 @@ class Sampled:
         return r
 
 
-def run(name, steps=None):
+def run(name, steps=None, queued=False):
     cfg = W.get(name)
     s = Sampled(cfg)
-    out = [s.step(k) for k in range(1, (steps or cfg.steps) + 1)]
+    out = [s.step(k, queued) for k in range(1, (steps or cfg.steps) + 1)]
     s.opt.close()
     return out
 
@@ -142,6 +147,13 @@ def test_fullsize_gpt2_medium_dynamic_scale_and_clip():
     rs = run("gpt2_medium")
     assert any(r["found_inf"] for r in rs)           # S grows until it overflows
     assert any(r["clipped"] for r in rs)
+
+
+def test_fullsize_gpt2_medium_queued_steps():
+    """The benchmark's launch configuration: mpt_step_async with S kept on the
+    device, default bins, full list."""
+    rs = run("gpt2_medium", steps=16, queued=True)
+    assert any(r["found_inf"] for r in rs)           # S reaches 2^18-2^19 by step 9-13
 
 
 def test_fullsize_gpt_1p3b():

@@ -262,6 +262,42 @@ def test_stats_and_timing():
 # queued (asynchronous) steps with the loss scale kept on the device
 # ---------------------------------------------------------------------------
 
+def test_cuda_graph_replays_follow_the_oracle():
+    """One queued step captured into a CUDA graph and replayed: the gradient
+    pointers are those of the step before, so the capture holds the two
+    kernel launches only (no pointer-table copy); each replay reads and
+    advances the device scale state and the gradients the buffers hold at
+    replay time.  Every replay must match the oracle, overflow steps too."""
+    plan = {4: [(1, 7, 0x7C00)]}
+    cfg = custom([60_000, 1031, 5, 40_000], law=("log2_uniform", -26.0, -2.0), scale0=2.0 ** 12,
+                 growth_interval=2, clip=0.3, steps=8, injections=lambda s: plan.get(s, []))
+    p = Pair(cfg)
+    p.step()                                   # uploads the pointer table of p.gviews
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=side):
+        p.opt.step_async(p.gviews, cfg.lr, cfg.momentum, cfg.weight_decay, cfg.clip, stream=side)
+    torch.cuda.synchronize()
+    skipped = 0
+    for _ in range(5):
+        p.step_no += 1
+        host = p.grads(p.step_no, p.scale)
+        p.flat.copy_(host)
+        torch.cuda.synchronize()
+        graph.replay()
+        r = p.opt.wait()
+        hv = [v.numpy().view(np.uint16) for v in p.layout.views(host)]
+        ro = oracle.step(p.state, hv, p.scale, cfg.lr, cfg.momentum, cfg.weight_decay,
+                         clip=cfg.clip, cfg=p.ocfg, flags=p.oflags, eps=p.eps)
+        p.compare_result(r, ro)
+        p.compare_state(f"replay {p.step_no}", exact=(r["clip_coef"] == ro["clip_coef"]))
+        p.scale = r["new_scale"]
+        skipped += r["found_inf"]
+    assert skipped == 1
+    del graph
+
+
 def test_async_steps_follow_the_oracle():
     """Steps queued back to back with mpt_step_async: S is read from and
     advanced on the device; each step's gradients are drawn at the S the
