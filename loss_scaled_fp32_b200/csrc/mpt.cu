@@ -2,10 +2,11 @@
 //
 // One step = two kernel launches on the caller's stream and, for the
 // waiting call, one 384-byte read-back of the control block:
-//   check_kernel  (2 B/param)  overflow flag, range counts, sum of squares,
-//                              last-CTA finish -> norm, clip coefficient
-//   update_kernel (20 B/param) fused unscale/clip/decay/momentum/master/FP16,
-//                              or counting only when the step overflowed
+//   check_kernel  (2 B/param)  overflow flag, sum of squares, two-level
+//                              finish -> norm, clip coefficient, next S
+//   update_kernel (20 B/param) fused unscale/clip/decay/momentum/master/FP16
+//                              and range counts; on an overflow step only a
+//                              counting sweep by its first CTAs
 // The launch order alone carries the check result to the update, so no host
 // decision sits between the two kernels.  The loss-scale state machine runs in
 // the check kernel's last CTA and keeps S on the device, so that steps can be
