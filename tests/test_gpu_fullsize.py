@@ -26,7 +26,7 @@ import torch
 
 import oracle
 import workloads as W
-from loss_scaled_fp32_b200 import MPT, Config
+from loss_scaled_fp32_b200 import MPT, Config, MPT_FLAG_GRAD_STATS, MPT_SCALER_DIRECT
 
 pytestmark = pytest.mark.gpu
 
@@ -34,7 +34,7 @@ THREADS = min(16, os.cpu_count() or 1)
 
 
 class Sampled:
-    def __init__(self, cfg, n_random=200_000, seed=0):
+    def __init__(self, cfg, n_random=200_000, seed=0, mpt_kw=None, ocfg_kw=None):
         self.cfg = cfg
         sizes = np.array(cfg.sizes, dtype=np.int64)
         starts = np.concatenate([[0], np.cumsum(sizes)[:-1]])
@@ -44,8 +44,11 @@ class Sampled:
         self.tensor = np.searchsorted(starts, idx, side="right") - 1
         self.elem = idx - starts[self.tensor]
         self.layout = W.GradLayout(cfg.sizes)
+        mpt_kw = mpt_kw or {}
         self.opt = MPT(cfg.sizes, Config(backoff=cfg.backoff, growth=cfg.growth,
-                                         growth_interval=cfg.growth_interval))
+                                         growth_interval=cfg.growth_interval, **mpt_kw))
+        self.hist = bool(mpt_kw.get("flags", 0) & MPT_FLAG_GRAD_STATS)
+        self.stats = self.hist or mpt_kw.get("scaler_mode", 0) == MPT_SCALER_DIRECT
         for i, m in enumerate(W.make_master(cfg, "cuda")):
             self.opt.master(i).copy_(m)
         self.opt.refresh_half()
@@ -64,7 +67,7 @@ class Sampled:
         self.w, self.v, self.h = m, v, h
         self.grad_idx = torch.from_numpy(np.array(self.layout.offsets)[self.tensor] + self.elem).cuda()
         self.ocfg = oracle.scaler_cfg(backoff=cfg.backoff, growth=cfg.growth,
-                                      growth_interval=cfg.growth_interval)
+                                      growth_interval=cfg.growth_interval, **(ocfg_kw or {}))
         self.scale = cfg.scale0
         self.clean = 0
         self.flat = torch.zeros(self.layout.total, dtype=torch.int16, device="cuda")
@@ -91,6 +94,10 @@ class Sampled:
             total.n_subnormal += r.n_subnormal
             total.n_nonfinite += r.n_nonfinite
             total.sumsq += r.sumsq
+            total.max_mag16 = max(total.max_mag16, r.max_mag16)
+            total.max_abs = max(total.max_abs, r.max_abs)
+            for b in range(32):
+                total.exp_hist[b] += r.exp_hist[b]
         return total
 
     def step(self, k, queued=False):
@@ -107,8 +114,13 @@ class Sampled:
         ro = oracle.clip_coef(self.full_check(self.scale), cfg.clip)
         for key in ("found_inf", "clipped", "n_zero", "n_subnormal", "n_nonfinite"):
             assert r[key] == getattr(ro, key), (k, key, r[key], getattr(ro, key))
-        new_scale, self.clean = oracle.scaler_next(self.ocfg, ro.found_inf, self.scale, self.clean)
+        new_scale, self.clean = oracle.scaler_next(self.ocfg, ro.found_inf, self.scale, self.clean,
+                                                   ro.max_abs)
         assert r["new_scale"] == new_scale and r["clean_run"] == self.clean, k
+        if self.stats:
+            assert r["max_abs_grad"] == ro.max_abs, (k, r["max_abs_grad"], ro.max_abs)
+        if self.hist:
+            assert self.opt.grad_histogram() == list(ro.exp_hist), k
         if ro.found_inf:
             assert math.isinf(r["grad_norm"])
         else:
@@ -130,9 +142,9 @@ class Sampled:
         return r
 
 
-def run(name, steps=None, queued=False):
+def run(name, steps=None, queued=False, **kw):
     cfg = W.get(name)
-    s = Sampled(cfg)
+    s = Sampled(cfg, **kw)
     out = [s.step(k, queued) for k in range(1, (steps or cfg.steps) + 1)]
     s.opt.close()
     return out
@@ -154,6 +166,17 @@ def test_fullsize_gpt2_medium_queued_steps():
     device, default bins, full list."""
     rs = run("gpt2_medium", steps=16, queued=True)
     assert any(r["found_inf"] for r in rs)           # S reaches 2^18-2^19 by step 9-13
+
+
+def test_fullsize_gpt2_medium_direct_scale_and_statistics():
+    """Direct scaler mode (S from each step's largest gradient, so S is not a
+    power of two: the check pass takes its binary32-product route) with the
+    exponent histogram, over the full list: the largest magnitude, the
+    histogram and each next S exact."""
+    rs = run("gpt2_medium", steps=6,
+             mpt_kw=dict(scaler_mode=MPT_SCALER_DIRECT, flags=MPT_FLAG_GRAD_STATS),
+             ocfg_kw=dict(mode=oracle.SCALER_DIRECT))
+    assert any(math.frexp(r["new_scale"])[0] != 0.5 for r in rs)
 
 
 def test_fullsize_gpt_1p3b():
