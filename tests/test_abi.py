@@ -84,44 +84,29 @@ def test_workspace_bytes():
     assert ws([10_000_000], check_chunk_elems=2048)[1] > ws([10_000_000])[1]
 
 
-def test_invalid_handles_and_arguments_return_codes():
+def test_default_check_bins_follow_the_list_size():
+    """Default check bins: 64K elements, halved (to 2048 at least) while the
+    list would give fewer than 296 bins.  Only the check table's size depends
+    on the chunk, so the explicit chunk whose workspace equals the default's
+    is the one the default chose; its neighbours differ by hundreds of bins,
+    which the 256-byte region rounding cannot hide."""
+    import workloads as W
     L = lsf.lib()
-    r = lsf.StepResult()
-    assert L.mpt_step(None, None, 1.0, 0.1, 0.9, 0.0, 0.0, None, ctypes.byref(r)) == lsf.MPT_ERR_INVALID_ARG
-    assert L.mpt_refresh_half(None, None) == lsf.MPT_ERR_INVALID_ARG
-    assert L.mpt_stats(None, ctypes.byref(lsf.Stats())) == lsf.MPT_ERR_INVALID_ARG
-    assert L.mpt_set_scaler_state(None, 1.0, 0) == lsf.MPT_ERR_INVALID_ARG
-    assert L.mpt_set_timing(None, 1) == lsf.MPT_ERR_INVALID_ARG
-    assert L.mpt_set_timing(None, -1) == lsf.MPT_ERR_INVALID_ARG
-    assert L.mpt_destroy(None) == 0
-    sizes = (ctypes.c_int64 * 1)(100)
-    h = ctypes.c_void_p()
-    # host memory is not a device workspace (and there may be no device at all)
-    buf = ctypes.create_string_buffer(1 << 16)
-    rc = L.mpt_create(sizes, 1, None, ctypes.c_void_p(ctypes.addressof(buf)), 1 << 16, ctypes.byref(h))
-    assert rc in (lsf.MPT_ERR_WORKSPACE, lsf.MPT_ERR_CUDA) and not h.value
-    # too small / misaligned workspace is rejected before any CUDA call
-    rc = L.mpt_create(sizes, 1, None, ctypes.c_void_p(256), 16, ctypes.byref(h))
-    assert rc == lsf.MPT_ERR_WORKSPACE
-    rc = L.mpt_create(sizes, 1, None, ctypes.c_void_p(ctypes.addressof(buf) | 8), 1 << 16, ctypes.byref(h))
-    assert rc == lsf.MPT_ERR_WORKSPACE
 
+    def ws(sizes, **cfg):
+        arr = (ctypes.c_int64 * len(sizes))(*sizes)
+        nb = ctypes.c_size_t()
+        assert L.mpt_workspace_bytes(arr, len(sizes), ctypes.byref(lsf.Config(**cfg)),
+                                     ctypes.byref(nb)) == 0
+        return nb.value
 
-def test_error_strings():
-    L = lsf.lib()
-    for code in (0, -1, -2, -3, -4, -5, 17):
-        s = L.mpt_error_string(code)
-        assert isinstance(s, bytes) and len(s) > 0
-
-
-def test_binding_fails_loudly_without_the_library(tmp_path, monkeypatch):
-    import importlib
-    monkeypatch.setattr(mbuild, "LIB", str(tmp_path / "absent" / "libmpt.so"))
-
-    def no_nvcc():
-        raise RuntimeError("nvcc not found: libmpt cannot be built")
-    monkeypatch.setattr(mbuild, "nvcc", no_nvcc)
-    monkeypatch.setattr(lsf, "_LIB", None)
-    with pytest.raises(RuntimeError):
-        lsf.lib()
-    monkeypatch.setattr(lsf, "_LIB", None)
+    cases = [([1 << 20], 2048),                    # 512 bins; 4K would give 256
+             ([10_000_000], 32768),                # 306 bins; 64K would give 153
+             ([19_300_000], 32768),                # 64K gives 295 < 296: halved
+             (W.get("resnet50").sizes, 65536)]     # 390 bins of 64K
+    for sizes, chunk in cases:
+        assert ws(sizes) == ws(sizes, check_chunk_elems=chunk), (sizes[:2], chunk)
+        for other in (chunk // 2, chunk * 2):
+            if 2048 <= other <= 65536:
+                assert ws(sizes, check_chunk_elems=other) != ws(sizes), (sizes[:2], other)
+    assert ws([5000]) == ws([5000], check_chunk_elems=2048)   # nothing below 2048
