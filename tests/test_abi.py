@@ -110,3 +110,46 @@ def test_default_check_bins_follow_the_list_size():
             if 2048 <= other <= 65536:
                 assert ws(sizes, check_chunk_elems=other) != ws(sizes), (sizes[:2], other)
     assert ws([5000]) == ws([5000], check_chunk_elems=2048)   # nothing below 2048
+
+
+def test_invalid_handles_and_arguments_return_codes():
+    L = lsf.lib()
+    r = lsf.StepResult()
+    assert L.mpt_step(None, None, 1.0, 0.1, 0.9, 0.0, 0.0, None, ctypes.byref(r)) == lsf.MPT_ERR_INVALID_ARG
+    assert L.mpt_refresh_half(None, None) == lsf.MPT_ERR_INVALID_ARG
+    assert L.mpt_stats(None, ctypes.byref(lsf.Stats())) == lsf.MPT_ERR_INVALID_ARG
+    assert L.mpt_set_scaler_state(None, 1.0, 0) == lsf.MPT_ERR_INVALID_ARG
+    assert L.mpt_set_timing(None, 1) == lsf.MPT_ERR_INVALID_ARG
+    assert L.mpt_set_timing(None, -1) == lsf.MPT_ERR_INVALID_ARG
+    assert L.mpt_destroy(None) == 0
+    sizes = (ctypes.c_int64 * 1)(100)
+    h = ctypes.c_void_p()
+    # host memory is not a device workspace (and there may be no device at all)
+    buf = ctypes.create_string_buffer(1 << 16)
+    rc = L.mpt_create(sizes, 1, None, ctypes.c_void_p(ctypes.addressof(buf)), 1 << 16, ctypes.byref(h))
+    assert rc in (lsf.MPT_ERR_WORKSPACE, lsf.MPT_ERR_CUDA) and not h.value
+    # too small / misaligned workspace is rejected before any CUDA call
+    rc = L.mpt_create(sizes, 1, None, ctypes.c_void_p(256), 16, ctypes.byref(h))
+    assert rc == lsf.MPT_ERR_WORKSPACE
+    rc = L.mpt_create(sizes, 1, None, ctypes.c_void_p(ctypes.addressof(buf) | 8), 1 << 16, ctypes.byref(h))
+    assert rc == lsf.MPT_ERR_WORKSPACE
+
+
+def test_error_strings():
+    L = lsf.lib()
+    for code in (0, -1, -2, -3, -4, -5, 17):
+        s = L.mpt_error_string(code)
+        assert isinstance(s, bytes) and len(s) > 0
+
+
+def test_binding_fails_loudly_without_the_library(tmp_path, monkeypatch):
+    import importlib
+    monkeypatch.setattr(mbuild, "LIB", str(tmp_path / "absent" / "libmpt.so"))
+
+    def no_nvcc():
+        raise RuntimeError("nvcc not found: libmpt cannot be built")
+    monkeypatch.setattr(mbuild, "nvcc", no_nvcc)
+    monkeypatch.setattr(lsf, "_LIB", None)
+    with pytest.raises(RuntimeError):
+        lsf.lib()
+    monkeypatch.setattr(lsf, "_LIB", None)
