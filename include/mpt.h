@@ -312,6 +312,15 @@ int mpt_set_scaler_state(mpt_handle* h, float scale, int32_t clean_run);
  * Errors: MPT_ERR_INVALID_ARG (h NULL, every < 0), MPT_ERR_CUDA. */
 int mpt_set_timing(mpt_handle* h, int32_t every);
 
+/* Test hook (the pages have no counterpart): the next step of this handle --
+ * mpt_step, mpt_step_async, mpt_step_partial or mpt_step_finish -- fails as
+ * if its kernel launch had failed: it queues nothing, returns MPT_ERR_CUDA,
+ * and the handle becomes unusable (every later call returns MPT_ERR_BROKEN),
+ * exactly as after a real CUDA error.  No CUDA call is made and no GPU fault
+ * is involved; it exists so that a caller's error path can be tested.
+ * Errors: MPT_ERR_INVALID_ARG (h NULL). */
+int mpt_debug_fail_next_step(mpt_handle* h);
+
 /* Release the handle's host resources.  The workspace is the caller's and is
  * not freed.  NULL is accepted. */
 int mpt_destroy(mpt_handle* h);

@@ -133,6 +133,7 @@ def lib():
             "mpt_shard_len": [ctypes.c_int64, i32, ctypes.POINTER(ctypes.c_int64)],
             "mpt_step_partial": [vp, vp, vp, ctypes.POINTER(vp)],
             "mpt_step_finish": [vp, vp, i32, f32, f32, f32, f32, vp],
+            "mpt_debug_fail_next_step": [vp],
         }
         for name, args in sig.items():
             fn = getattr(L, name)
@@ -321,6 +322,11 @@ class MPT:
         """Time the two kernels of every ``every``-th following step (0 or
         False: off; True or 1: every step)."""
         _check(lib().mpt_set_timing(self._h, int(every)), "mpt_set_timing")
+
+    def debug_fail_next_step(self):
+        """Test hook: the next step fails like a failed kernel launch and the
+        handle becomes unusable (``mpt_debug_fail_next_step``)."""
+        _check(lib().mpt_debug_fail_next_step(self._h), "mpt_debug_fail_next_step")
 
     def close(self):
         if getattr(self, "_h", None):

@@ -12,6 +12,7 @@
 // the check kernel's last CTA and keeps S on the device, so that steps can be
 // queued without waiting (mpt_step_async); the host mirrors it on read-back.
 #include <cuda_runtime.h>
+#include <nvtx3/nvToolsExt.h>
 
 #include <cmath>
 #include <cstdlib>
@@ -253,6 +254,7 @@ struct mpt_handle {
     int32_t clean_run = 0;
     mpt_stats_t stats{};
     bool broken = false;
+    bool fail_next = false;              // test hook: the next step fails as a launch would
     // kernel timing: ring of (start, between, end) events, one per timed step;
     // every timing_every-th step queued since mpt_set_timing is timed
     int32_t timing_every = 0;
@@ -391,6 +393,15 @@ static void launch_update_any(const mpt_handle* h, const UpdateArgs& ua, bool st
 // followed by the update).
 enum class Phase { kWhole, kShardCheck, kShardFinish };
 
+// An NVTX range around the host work of one call (named ranges for a
+// timeline profiler; near-free when no tool is attached).
+struct NvtxRange {
+    explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+    ~NvtxRange() { nvtxRangePop(); }
+    NvtxRange(const NvtxRange&) = delete;
+    NvtxRange& operator=(const NvtxRange&) = delete;
+};
+
 // Queue a step (or a phase of a sharded step) on st.  scale_on_device: S
 // comes from the device scale state instead of host_scale.
 static int enqueue_step(mpt_handle* h, const void* const* d_grads_half, bool scale_on_device,
@@ -398,12 +409,19 @@ static int enqueue_step(mpt_handle* h, const void* const* d_grads_half, bool sca
                         float clip, cudaStream_t st, Phase phase = Phase::kWhole,
                         const void* d_parts = nullptr, int32_t world = 0)
 {
+    NvtxRange range(phase == Phase::kWhole ? "mpt.step" :
+                    phase == Phase::kShardCheck ? "mpt.step_partial" : "mpt.step_finish");
     if (phase == Phase::kShardFinish)
         d_grads_half = h->last_ptrs.data();  // the pointers of the check pass
     for (int32_t i = 0; i < h->n; ++i) {
         const uintptr_t p = reinterpret_cast<uintptr_t>(d_grads_half[i]);
         if (p == 0 || (p & 1))
             return MPT_ERR_INVALID_ARG;
+    }
+    if (h->fail_next) {
+        // test hook: report what a failed kernel launch reports, queue nothing
+        h->fail_next = false;
+        return MPT_ERR_CUDA;
     }
     const size_t ptr_bytes = sizeof(void*) * (size_t)h->n;
 
@@ -798,6 +816,7 @@ int mpt_step_finish(mpt_handle* h, const void* d_partials, int32_t world, float 
 
 int mpt_wait(mpt_handle* h, void* cuda_stream, mpt_step_result* out)
 {
+    NvtxRange range("mpt.wait");
     if (!h)
         return MPT_ERR_INVALID_ARG;
     if (h->broken)
@@ -875,6 +894,14 @@ int mpt_set_timing(mpt_handle* h, int32_t every)
     }
     h->timing_every = every;
     h->timing_count = 0;
+    return MPT_OK;
+}
+
+int mpt_debug_fail_next_step(mpt_handle* h)
+{
+    if (!h)
+        return MPT_ERR_INVALID_ARG;
+    h->fail_next = true;
     return MPT_OK;
 }
 

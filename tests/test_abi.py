@@ -121,6 +121,7 @@ def test_invalid_handles_and_arguments_return_codes():
     assert L.mpt_set_scaler_state(None, 1.0, 0) == lsf.MPT_ERR_INVALID_ARG
     assert L.mpt_set_timing(None, 1) == lsf.MPT_ERR_INVALID_ARG
     assert L.mpt_set_timing(None, -1) == lsf.MPT_ERR_INVALID_ARG
+    assert L.mpt_debug_fail_next_step(None) == lsf.MPT_ERR_INVALID_ARG
     assert L.mpt_destroy(None) == 0
     sizes = (ctypes.c_int64 * 1)(100)
     h = ctypes.c_void_p()

@@ -159,6 +159,60 @@ def test_huge_inverse_scale_overflows_products_not_the_check():
     p.compare_state("huge 1/S", exact=True)
 
 
+def test_steps_write_nothing_outside_the_tensors():
+    """Guard canaries: every byte of the master, momentum and FP16 arenas that
+    belongs to no tensor (the 16-element padding after each tensor and the
+    alignment gaps between the arenas) is filled with a pattern after the FP16
+    refresh; steps over chunk bins with ragged tails, packed bins, an
+    overflow step and a clipped step must leave every one of them intact."""
+    plan = {3: [(2, 100, 0x7C00)]}
+    sizes = [1, 17, 1025, 4097, 70_001, 3, 65_536 + 5, 1000]
+    cfg = custom(sizes, law=("log2_uniform", -26.0, -4.0), scale0=2.0 ** 12, growth_interval=2,
+                 clip=0.05, steps=5, injections=lambda s: plan.get(s, []))
+    p = Pair(cfg)
+    ws = p.opt.workspace
+    base = ws.data_ptr()
+    spans = []
+    for i in range(len(sizes)):
+        for t in (p.opt.master(i), p.opt.momentum(i), p.opt.w16(i)):
+            spans.append((t.data_ptr() - base, t.data_ptr() - base + t.numel() * t.element_size()))
+    spans.sort()
+    gaps = [(a_end, b_start) for (_, a_end), (b_start, _) in zip(spans, spans[1:]) if b_start > a_end]
+    tail = (spans[-1][1], (spans[-1][1] + 31) // 32 * 32)       # the last tensor's padding
+    if tail[1] > tail[0]:
+        gaps.append(tail)
+    assert len(gaps) >= len(sizes)                                # at least one per tensor
+    idx = torch.cat([torch.arange(a, b, device="cuda") for a, b in gaps])
+    pattern = (torch.arange(idx.numel(), device="cuda") * 37 % 251 + 3).to(torch.uint8)
+    ws[idx] = pattern
+    torch.cuda.synchronize()
+    for _ in range(cfg.steps):
+        p.step()
+    assert p.bitexact_steps >= 3
+    assert torch.equal(ws[idx], pattern)
+
+
+def test_injected_launch_failure_breaks_the_handle():
+    """The test hook makes the next step fail as a failed kernel launch would
+    (no CUDA call, no GPU fault): MPT_ERR_CUDA, then MPT_ERR_BROKEN for every
+    later call; the handle can still be destroyed."""
+    from loss_scaled_fp32_b200 import MptError
+    cfg = custom([5000, 33], steps=2)
+    p = Pair(cfg)
+    p.step()
+    p.opt.debug_fail_next_step()
+    with pytest.raises(MptError) as e:
+        p.opt.step(p.gviews, p.scale, cfg.lr, cfg.momentum, cfg.weight_decay)
+    assert e.value.code == -3                                     # MPT_ERR_CUDA
+    for call in (lambda: p.opt.step(p.gviews, p.scale, cfg.lr, cfg.momentum, cfg.weight_decay),
+                 lambda: p.opt.step_async(p.gviews, cfg.lr, cfg.momentum, cfg.weight_decay),
+                 lambda: p.opt.wait()):
+        with pytest.raises(MptError) as e:
+            call()
+        assert e.value.code == -5                                 # MPT_ERR_BROKEN
+    p.opt.close()
+
+
 def test_checked_mode_and_stale_counts():
     cfg = custom([100_000, 17, 3000], steps=3, lr=1e-3)
     p = Pair(cfg, flags=MPT_FLAG_CHECKED | MPT_FLAG_COUNT_STALE)
