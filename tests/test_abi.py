@@ -154,3 +154,24 @@ def test_binding_fails_loudly_without_the_library(tmp_path, monkeypatch):
     with pytest.raises(RuntimeError):
         lsf.lib()
     monkeypatch.setattr(lsf, "_LIB", None)
+
+def test_plain_c_consumer_compiles_links_and_runs(tmp_path):
+    """The header is strict C99 and the library links from C: a plain C
+    program takes the address of every declared entry point and runs the
+    calls that need no GPU (tests/native/abi_consumer.c)."""
+    import shutil
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("no gcc")
+    lib_path = lsf.lib()._name
+    lib_dir = os.path.dirname(lib_path)
+    exe = str(tmp_path / "abi_consumer")
+    build = subprocess.run(
+        [gcc, "-std=c99", "-Wall", "-Wextra", "-Wpedantic", "-Werror",
+         "-I", os.path.join(ROOT, "include"), os.path.join(ROOT, "tests", "native", "abi_consumer.c"),
+         "-L", lib_dir, "-lmpt", "-Wl,-rpath," + lib_dir, "-o", exe],
+        capture_output=True, text=True)
+    assert build.returncode == 0, build.stderr
+    run = subprocess.run([exe], capture_output=True, text=True, timeout=120)
+    assert run.returncode == 0, run.stderr
+    assert "21 entry points" in run.stdout
