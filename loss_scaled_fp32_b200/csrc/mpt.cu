@@ -2,11 +2,12 @@
 //
 // One step = two kernel launches on the caller's stream and, for the
 // waiting call, one 384-byte read-back of the control block:
-//   check_kernel  (2 B/param)  overflow flag, sum of squares, two-level
-//                              finish -> norm, clip coefficient, next S
+//   check_kernel  (2 B/param)  overflow flag, sum of squares, range counts,
+//                              two-level finish -> norm, clip coefficient,
+//                              next S
 //   update_kernel (20 B/param) fused unscale/clip/decay/momentum/master/FP16
-//                              and range counts; on an overflow step only a
-//                              counting sweep by its first CTAs
+//                              over a persistent grid; on an overflow step
+//                              each CTA reads the flag and exits
 // The launch order alone carries the check result to the update, so no host
 // decision sits between the two kernels.  The loss-scale state machine runs in
 // the check kernel's last CTA and keeps S on the device, so that steps can be
@@ -14,6 +15,8 @@
 #include <cuda_runtime.h>
 #include <nvtx3/nvToolsExt.h>
 
+#include <algorithm>
+#include <atomic>
 #include <cmath>
 #include <cstdlib>
 #include <cstddef>
@@ -29,7 +32,7 @@
 using namespace mpt;
 
 static_assert(sizeof(Ctrl) == 384, "the control block read back each step is 384 bytes");
-static_assert(offsetof(Ctrl, zero_acc) == 128 && offsetof(Ctrl, sumsq) == 256,
+static_assert(offsetof(Ctrl, stale_acc) == 128 && offsetof(Ctrl, sumsq) == 256,
               "one 128-byte line per group of control fields");
 
 namespace {
@@ -242,6 +245,7 @@ struct mpt_handle {
     float* d_master = nullptr;
     float* d_momentum = nullptr;
     uint16_t* d_w16 = nullptr;
+    int32_t upd_grid = 0;                // CTAs of the persistent update grid
     // host state
     std::vector<const void*> last_ptrs;
     bool ptrs_uploaded = false;
@@ -319,10 +323,10 @@ static bool stats_on(const mpt_handle* h) { return stats_level(h) != kNoStats; }
 // dependent launch): its CTAs take the SMs the check CTAs free, load their
 // work descriptors, then wait for the check result (griddepcontrol.wait).
 template <int kOpt, bool kStale, bool kChecked>
-static void launch_update(const UpdateArgs& a, cudaStream_t st)
+static void launch_update(const UpdateArgs& a, int grid, cudaStream_t st)
 {
     cudaLaunchConfig_t lc = {};
-    lc.gridDim = dim3((unsigned int)a.t.nbins);
+    lc.gridDim = dim3((unsigned int)grid);
     lc.blockDim = dim3(kThreads);
     lc.dynamicSmemBytes = 0;
     lc.stream = st;
@@ -335,12 +339,46 @@ static void launch_update(const UpdateArgs& a, cudaStream_t st)
 }
 
 template <int kOpt>
-static void launch_update_opt(const UpdateArgs& a, bool stale, bool checked, cudaStream_t st)
+static void launch_update_opt(const UpdateArgs& a, int grid, bool stale, bool checked, cudaStream_t st)
 {
     if (stale)
-        checked ? launch_update<kOpt, true, true>(a, st) : launch_update<kOpt, true, false>(a, st);
+        checked ? launch_update<kOpt, true, true>(a, grid, st) : launch_update<kOpt, true, false>(a, grid, st);
     else
-        checked ? launch_update<kOpt, false, true>(a, st) : launch_update<kOpt, false, false>(a, st);
+        checked ? launch_update<kOpt, false, true>(a, grid, st) : launch_update<kOpt, false, false>(a, grid, st);
+}
+
+// The update-kernel instantiation a handle launches (its optimizer and flags
+// are fixed at creation).
+template <int kOpt>
+static const void* update_fn_opt(bool stale, bool checked)
+{
+    if (stale)
+        return checked ? (const void*)update_kernel<kOpt, true, true> : (const void*)update_kernel<kOpt, true, false>;
+    return checked ? (const void*)update_kernel<kOpt, false, true> : (const void*)update_kernel<kOpt, false, false>;
+}
+
+static const void* update_fn(const mpt_config& c)
+{
+    const bool stale = (c.flags & MPT_FLAG_COUNT_STALE) != 0;
+    const bool checked = (c.flags & MPT_FLAG_CHECKED) != 0;
+    switch (c.optimizer) {
+    case MPT_OPT_NESTEROV: return update_fn_opt<kOptNesterov>(stale, checked);
+    case MPT_OPT_ADAGRAD: return update_fn_opt<kOptAdagrad>(stale, checked);
+    default: return update_fn_opt<kOptMomentum>(stale, checked);
+    }
+}
+
+// Persistent update grid: every resident slot of every SM (the occupancy of
+// the handle's instantiation), never more CTAs than bins.
+static bool size_update_grid(mpt_handle* h)
+{
+    int sms = 0, per_sm = 0;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, h->device) != cudaSuccess ||
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, update_fn(h->cfg), kThreads, 0) != cudaSuccess)
+        return false;
+    const int64_t slots = (int64_t)std::max(1, sms) * std::max(1, per_sm);
+    h->upd_grid = (int32_t)std::min<int64_t>(slots, (int64_t)h->L.bins_update.size());
+    return h->upd_grid > 0;
 }
 
 // What the check pass needs from S (the same values the device computes when
@@ -381,10 +419,11 @@ static void launch_check_level(const mpt_handle* h, const CheckArgs& ca, bool ch
 static void launch_update_any(const mpt_handle* h, const UpdateArgs& ua, bool stale, bool checked,
                               cudaStream_t st)
 {
+    const int g = h->upd_grid;
     switch (h->cfg.optimizer) {
-    case MPT_OPT_NESTEROV: launch_update_opt<kOptNesterov>(ua, stale, checked, st); break;
-    case MPT_OPT_ADAGRAD: launch_update_opt<kOptAdagrad>(ua, stale, checked, st); break;
-    default: launch_update_opt<kOptMomentum>(ua, stale, checked, st); break;
+    case MPT_OPT_NESTEROV: launch_update_opt<kOptNesterov>(ua, g, stale, checked, st); break;
+    case MPT_OPT_ADAGRAD: launch_update_opt<kOptAdagrad>(ua, g, stale, checked, st); break;
+    default: launch_update_opt<kOptMomentum>(ua, g, stale, checked, st); break;
     }
 }
 
@@ -486,8 +525,6 @@ static int enqueue_step(mpt_handle* h, const void* const* d_grads_half, bool sca
     ua.mu = momentum;
     ua.wd = weight_decay;
     ua.eps = h->cfg.eps;
-    ua.check_bins = h->d_bins_check;
-    ua.check_nbins = (int32_t)h->L.bins_check.size();
 
     const bool checked = (h->cfg.flags & MPT_FLAG_CHECKED) != 0;
     const bool stale = (h->cfg.flags & MPT_FLAG_COUNT_STALE) != 0;
@@ -551,8 +588,8 @@ static int read_result(mpt_handle* h, cudaStream_t st, mpt_step_result* out)
     r.clipped = c.clipped;
     r.grad_norm = c.norm;
     r.clip_coef = c.coef;
-    r.n_zero = c.zero_acc;
-    r.n_subnormal = c.subnormal_acc;
+    r.n_zero = c.n_zero;
+    r.n_subnormal = c.n_subnormal;
     r.n_nonfinite = c.n_nonfinite;
     r.n_fp16_stale = stale ? c.stale_acc : 0;
     r.new_scale = c.scale;
@@ -564,8 +601,8 @@ static int read_result(mpt_handle* h, cudaStream_t st, mpt_step_result* out)
             h->hist[k] = h->hist_box[k];
     h->scale = c.scale;
     h->clean_run = c.clean_run;
-    if (c.steps_total > h->stats.steps)
-        h->stats.n_fp16_stale_total += r.n_fp16_stale;
+    // every step's stale count, queued steps included, is summed on the device
+    h->stats.n_fp16_stale_total = stale ? c.stale_total + c.stale_acc : 0;
     h->stats.steps = c.steps_total;
     h->stats.skipped = c.skipped_total;
     h->stats.scale = h->scale;
@@ -693,6 +730,7 @@ int mpt_create(const int64_t* sizes, int32_t n, const mpt_config* cfg, void* d_w
               cudaHostAlloc(reinterpret_cast<void**>(&h->hist_box), sizeof(h->hist), cudaHostAllocDefault) == cudaSuccess &&
               cudaEventCreateWithFlags(&h->ptrs_copied, cudaEventDisableTiming) == cudaSuccess &&
               upload_scaler_state(h, 1.0f, 0) &&
+              size_update_grid(h) &&
               cudaDeviceSynchronize() == cudaSuccess;
     if (!ok) {
         cudaGetLastError();
@@ -953,10 +991,11 @@ struct NoAllocCtrl {
 static_assert(sizeof(NoAllocCtrl) <= kNoAllocCtrlBytes, "counters fit their slot");
 static_assert(MPT_NOALLOC_MAX_ELEMS % kNoAllocChunk == 0, "whole bins");
 
-// Host-side lookup of the scratch array's device address, once per device.
-std::once_flag g_noalloc_once[kNoAllocMaxDevices];
-unsigned char* g_noalloc_addr[kNoAllocMaxDevices];
-cudaError_t g_noalloc_status[kNoAllocMaxDevices];
+// Host-side lookup of the scratch array's device address, per device: only a
+// successful lookup is kept, so a call that failed (say, inside a stream
+// capture) leaves the next call free to try again.
+std::mutex g_noalloc_mu;
+std::atomic<unsigned char*> g_noalloc_addr[kNoAllocMaxDevices];
 
 }  // namespace
 
@@ -982,7 +1021,7 @@ check_flat_kernel(const uint16_t* g, int64_t n, unsigned char* scratch, mpt_chec
     a.sq_unscale = sq_unscale;
     a.pow2 = kPow2;
     SqAcc s;
-    check_range<kPow2>(g + begin, len, a, s);
+    check_range<kPow2, false, kNoStats>(g + begin, len, a, s, nullptr, nullptr);
 
     unsigned int nf = 0;
     if (__syncthreads_or(s.saw_nonfinite())) {
@@ -1023,6 +1062,33 @@ check_flat_kernel(const uint16_t* g, int64_t n, unsigned char* scratch, mpt_chec
     }
 }
 
+// Set-up of one device, with that device current: the device address of the
+// scratch array (in host code its name is only a host-side stand-in) and the
+// loading of both kernel instantiations, so that no later call has to load a
+// module (under lazy loading that could otherwise happen inside a capture).
+static int noalloc_scratch(int dev, unsigned char** out)
+{
+    unsigned char* p = g_noalloc_addr[dev].load(std::memory_order_acquire);
+    if (!p) {
+        std::lock_guard<std::mutex> lock(g_noalloc_mu);
+        p = g_noalloc_addr[dev].load(std::memory_order_relaxed);
+        if (!p) {
+            void* addr = nullptr;
+            cudaFuncAttributes fa;
+            if (cudaGetSymbolAddress(&addr, g_noalloc_scratch) != cudaSuccess || !addr ||
+                cudaFuncGetAttributes(&fa, check_flat_kernel<true>) != cudaSuccess ||
+                cudaFuncGetAttributes(&fa, check_flat_kernel<false>) != cudaSuccess) {
+                cudaGetLastError();  // this failure's own error; a later call retries
+                return MPT_ERR_CUDA;
+            }
+            p = static_cast<unsigned char*>(addr);
+            g_noalloc_addr[dev].store(p, std::memory_order_release);
+        }
+    }
+    *out = p;
+    return MPT_OK;
+}
+
 extern "C" int mpt_check_flat_noalloc(const void* d_grads_half, int64_t n, float scale,
                                       float clip, mpt_check_result* d_result,
                                       void* cuda_stream)
@@ -1043,16 +1109,13 @@ extern "C" int mpt_check_flat_noalloc(const void* d_grads_half, int64_t n, float
     }
     if (dev < 0 || dev >= kNoAllocMaxDevices)
         return MPT_ERR_CUDA;
-    // In host code the array's name is a host-side stand-in, not a device
-    // address: look the address up once per device, with that device current.
-    std::call_once(g_noalloc_once[dev], [dev] {
-        g_noalloc_status[dev] =
-            cudaGetSymbolAddress(reinterpret_cast<void**>(&g_noalloc_addr[dev]), g_noalloc_scratch);
-    });
-    if (g_noalloc_status[dev] != cudaSuccess || !g_noalloc_addr[dev])
+    unsigned char* scratch = nullptr;
+    if (noalloc_scratch(dev, &scratch) != MPT_OK)
         return MPT_ERR_CUDA;
-    unsigned char* scratch = g_noalloc_addr[dev];
 
+    // Each runtime call's own status is checked (not the thread's last-error
+    // state, which may hold an error the caller has yet to collect); only an
+    // error of this call is cleared.
     cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
     // the counters must start at zero whatever the previous call left
     if (cudaMemsetAsync(scratch, 0, kNoAllocCtrlBytes, st) != cudaSuccess) {
@@ -1065,11 +1128,16 @@ extern "C" int mpt_check_flat_noalloc(const void* d_grads_half, int64_t n, float
     const double sq_unscale = pow2 ? std::ldexp(1.0, -2 * (e2 - 1)) : 0.0;
     const unsigned int bins = (unsigned int)((n + kNoAllocChunk - 1) / kNoAllocChunk);
     const uint16_t* g = static_cast<const uint16_t*>(d_grads_half);
-    if (pow2)
-        check_flat_kernel<true><<<bins, kThreads, 0, st>>>(g, n, scratch, d_result, inv_scale, sq_unscale, clip);
-    else
-        check_flat_kernel<false><<<bins, kThreads, 0, st>>>(g, n, scratch, d_result, inv_scale, sq_unscale, clip);
-    if (cudaGetLastError() != cudaSuccess)
+    cudaLaunchConfig_t lc = {};
+    lc.gridDim = dim3(bins);
+    lc.blockDim = dim3(kThreads);
+    lc.stream = st;
+    const cudaError_t e =
+        pow2 ? cudaLaunchKernelEx(&lc, check_flat_kernel<true>, g, n, scratch, d_result, inv_scale, sq_unscale, clip)
+             : cudaLaunchKernelEx(&lc, check_flat_kernel<false>, g, n, scratch, d_result, inv_scale, sq_unscale, clip);
+    if (e != cudaSuccess) {
+        cudaGetLastError();
         return MPT_ERR_CUDA;
+    }
     return MPT_OK;
 }

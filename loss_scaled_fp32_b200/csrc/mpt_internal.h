@@ -66,12 +66,15 @@ struct __align__(128) Ctrl {
     unsigned int ticket;
     unsigned int error_acc;
     unsigned int max_mag_acc;  // statistics mode: largest finite |g16| (atomicMax)
-    unsigned int pad0[27];
-    // line 1: update-kernel accumulators (cleared by the check kernel's last CTA)
-    unsigned long long zero_acc;
-    unsigned long long subnormal_acc;
+    unsigned int pad0a;
+    unsigned long long zero_acc;       // FP16 gradients equal to +-0
+    unsigned long long subnormal_acc;  // FP16 gradients with 0 < |g16| < 2^-14
+    unsigned int pad0[22];
+    // line 1: update-kernel accumulators and its work counter (cleared by
+    // the check kernel's last CTA)
     unsigned long long stale_acc;
-    unsigned int pad1[26];
+    unsigned int upd_next;     // update bins claimed beyond each CTA's first
+    unsigned int pad1[29];
     // line 2: step result written by the check kernel's last CTA
     double sumsq;
     double norm;
@@ -98,6 +101,12 @@ struct __align__(128) Ctrl {
     double next_sq_unscale;
     float next_inv;
     unsigned int pad3;
+    // range counts of this step's gradients (from the check pass)
+    unsigned long long n_zero;
+    unsigned long long n_subnormal;
+    // stale counts of every update before the last one (the last update's
+    // count is still in stale_acc)
+    unsigned long long stale_total;
 };
 
 // What one rank's check pass contributes to a sharded step (32 bytes): its

@@ -2,11 +2,12 @@
 //
 //   check_kernel   one pass over the FP16 gradients: overflow check (Step 6 of
 //                  "The Integrated Training Procedure (Figure 1)"), sum of
-//                  squares of the unscaled gradients (global-L2 clip), with a
-//                  deterministic two-level finish that writes the step result
+//                  squares of the unscaled gradients (global-L2 clip), zero
+//                  and subnormal counts, with a deterministic two-level
+//                  finish that writes the step result
 //   update_kernel  the fused per-element update (Steps 5 and 7, weight decay,
-//                  clip, FP16 copy); on an overflow step its first CTAs only
-//                  count zero and subnormal gradients, the rest exit
+//                  clip, FP16 copy) over a persistent grid; on an overflow
+//                  step every CTA reads the flag and exits
 //   refresh_kernel FP16 copy = round-to-nearest-even(master) (Step 1)
 //
 // All three are HBM-bound streaming kernels on the CUDA cores: there is no
@@ -76,8 +77,6 @@ struct UpdateArgs {
     float mu;
     float wd;
     float eps;            // Adagrad only
-    const Bin* check_bins;  // the check pass's (larger) bins: the counting
-    int32_t check_nbins;    // sweep of an overflow step walks these
 };
 
 // What the squares need from S: the binary32 reciprocal 1/S and, when S is a
@@ -158,9 +157,12 @@ __device__ __forceinline__ void finish_step(Ctrl* c, float S, const SqParams& q,
     c->next_pow2 = nq.pow2 ? 1 : 0;
     c->clean_run = clean;
     c->steps_total += 1;
-    c->zero_acc = 0;
-    c->subnormal_acc = 0;
-    c->stale_acc = 0;
+    // range counts of this step's check pass; the previous update's stale
+    // count joins the running total; the update's accumulators start over
+    c->n_zero = atomicExch(&c->zero_acc, 0ull);
+    c->n_subnormal = atomicExch(&c->subnormal_acc, 0ull);
+    c->stale_total += atomicExch(&c->stale_acc, 0ull);
+    c->upd_next = 0;
 }
 
 
@@ -291,13 +293,6 @@ __device__ __forceinline__ void sq_vec(uint4 v, const SqParams& a, SqAcc& s)
     sq_word<kPow2>(v.w, a, s);
 }
 
-template <bool kPow2>
-__device__ __forceinline__ void sq_vec(uint2 v, const SqParams& a, SqAcc& s)
-{
-    sq_word<kPow2>(v.x, a, s);
-    sq_word<kPow2>(v.y, a, s);
-}
-
 // Statistics mode: each thread counts the binary16 exponent fields it sees in
 // its own row of a shared-memory table (rows padded to 33 words, so that
 // threads of a warp incrementing the same bin hit different banks) and keeps
@@ -343,75 +338,98 @@ __device__ __forceinline__ void stats_vec(uint4 v, StatsAcc* st)
     stats_word<kStats>(v.w, st);
 }
 
-template <int kStats>
-__device__ __forceinline__ void stats_vec(uint2 v, StatsAcc* st)
+// Range counts of the gradients (how many are +-0 and how many are
+// subnormal in binary16: the part of the gradient distribution that FP16
+// flushes or keeps only with reduced precision).  Lane-packed counters: each
+// 32-bit word carries two 16-bit counts, one per FP16 lane of a gradient
+// word; a thread adds at most 2^11 per lane (at most 2^20 elements per bin),
+// far below overflow.
+struct RangeCounts {
+    uint32_t nz2 = 0;  // lanes with |g16| != 0
+    uint32_t ns2 = 0;  // lanes with |g16| >= 2^-14 (normal, inf or NaN)
+
+    __device__ __forceinline__ void word(uint32_t w)
+    {
+        const uint32_t m = w & 0x7FFF7FFFu;
+        nz2 += ((m + 0x7FFF7FFFu) >> 15) & 0x00010001u;  // lane != +-0
+        ns2 += ((m + 0x7C007C00u) >> 15) & 0x00010001u;  // lane >= 2^-14
+    }
+    __device__ __forceinline__ void half(uint16_t h)
+    {
+        const uint32_t m = h & 0x7FFFu;
+        nz2 += m != 0 ? 1u : 0u;
+        ns2 += m >= 0x0400u ? 1u : 0u;
+    }
+    __device__ __forceinline__ unsigned int nonzero() const { return (nz2 & 0xFFFFu) + (nz2 >> 16); }
+    __device__ __forceinline__ unsigned int normal() const { return (ns2 & 0xFFFFu) + (ns2 >> 16); }
+};
+
+// Gradients of the check pass per thread: 16-B loads, kCheckVecs of them in
+// flight per thread (64 B).
+constexpr int kCheckVecs = 4;
+
+template <bool kPow2, bool kCount, int kStats>
+__device__ __forceinline__ void check_half(uint16_t h, const SqParams& a, SqAcc& s,
+                                           RangeCounts* rc, StatsAcc* st)
 {
-    stats_word<kStats>(v.x, st);
-    stats_word<kStats>(v.y, st);
+    sq_half<kPow2>(h, a, s);
+    if constexpr (kCount)
+        rc->half(h);
+    stats_half<kStats>(h, st);
 }
 
-// One contiguous range: 16-B loads when aligned, 8-B when 8-B aligned, else
-// 2-B loads; unrolled so that every thread has 64 B of loads in flight.
-template <bool kPow2, typename Vec, int kStats = kNoStats>
+// One contiguous range of gradients starting on a 16-byte boundary.
+template <bool kPow2, bool kCount, int kStats>
 __device__ __forceinline__ void check_range_vec(const uint16_t* g, int len, const SqParams& a,
-                                                SqAcc& s, StatsAcc* st = nullptr)
+                                                SqAcc& s, RangeCounts* rc, StatsAcc* st)
 {
-    constexpr int kPer = sizeof(Vec) / 2;
-    constexpr int kUnroll = 64 / sizeof(Vec);
-    const Vec* gv = reinterpret_cast<const Vec*>(g);
-    const int nv = len / kPer;
+    constexpr int kU = kCheckVecs;
+    const uint4* gv = reinterpret_cast<const uint4*>(g);
+    const int nv = len >> 3;
     int i = threadIdx.x;
-    for (; i + (kUnroll - 1) * kThreads < nv; i += kUnroll * kThreads) {
-        Vec v[kUnroll];
+    for (; i + (kU - 1) * kThreads < nv; i += kU * kThreads) {
+        uint4 v[kU];
 #pragma unroll
-        for (int k = 0; k < kUnroll; ++k)
+        for (int k = 0; k < kU; ++k)
             v[k] = __ldg(gv + i + k * kThreads);
 #pragma unroll
-        for (int k = 0; k < kUnroll; ++k) {
+        for (int k = 0; k < kU; ++k) {
             sq_vec<kPow2>(v[k], a, s);
+            if constexpr (kCount) {
+                rc->word(v[k].x);
+                rc->word(v[k].y);
+                rc->word(v[k].z);
+                rc->word(v[k].w);
+            }
             stats_vec<kStats>(v[k], st);
         }
     }
     for (; i < nv; i += kThreads) {
-        const Vec v = __ldg(gv + i);
+        const uint4 v = __ldg(gv + i);
         sq_vec<kPow2>(v, a, s);
+        if constexpr (kCount) {
+            rc->word(v.x);
+            rc->word(v.y);
+            rc->word(v.z);
+            rc->word(v.w);
+        }
         stats_vec<kStats>(v, st);
     }
-    for (int j = nv * kPer + threadIdx.x; j < len; j += kThreads) {
-        const uint16_t h = __ldg(g + j);
-        sq_half<kPow2>(h, a, s);
-        stats_half<kStats>(h, st);
-    }
+    for (int j = (nv << 3) + threadIdx.x; j < len; j += kThreads)
+        check_half<kPow2, kCount, kStats>(__ldg(g + j), a, s, rc, st);
 }
 
-template <bool kPow2, int kStats = kNoStats>
+// One contiguous range at any 2-byte alignment: the elements before the
+// first 16-byte boundary one per thread, the rest with 16-B loads.
+template <bool kPow2, bool kCount, int kStats>
 __device__ __forceinline__ void check_range(const uint16_t* g, int len, const SqParams& a,
-                                            SqAcc& s, StatsAcc* st = nullptr)
+                                            SqAcc& s, RangeCounts* rc, StatsAcc* st)
 {
     const uintptr_t p = reinterpret_cast<uintptr_t>(g);
-    if ((p & 15) == 0) {
-        check_range_vec<kPow2, uint4, kStats>(g, len, a, s, st);
-    } else if ((p & 7) == 0) {
-        check_range_vec<kPow2, uint2, kStats>(g, len, a, s, st);
-    } else {
-        int j = threadIdx.x;
-        for (; j + 3 * kThreads < len; j += 4 * kThreads) {
-            uint16_t h[4];
-#pragma unroll
-            for (int k = 0; k < 4; ++k)
-                h[k] = __ldg(g + j + k * kThreads);
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                sq_half<kPow2>(h[k], a, s);
-                stats_half<kStats>(h[k], st);
-            }
-        }
-        for (; j < len; j += kThreads) {
-            const uint16_t h = __ldg(g + j);
-            sq_half<kPow2>(h, a, s);
-            stats_half<kStats>(h, st);
-        }
-    }
+    const int head = min(len, (int)(((16u - (unsigned int)(p & 15u)) & 15u) >> 1));
+    if ((int)threadIdx.x < head)
+        check_half<kPow2, kCount, kStats>(__ldg(g + threadIdx.x), a, s, rc, st);
+    check_range_vec<kPow2, kCount, kStats>(g + head, len - head, a, s, rc, st);
 }
 
 // Fixed-shape block sum (result valid in thread 0): deterministic for a fixed
@@ -429,6 +447,40 @@ __device__ __forceinline__ double block_sum(double x, double* red)
 #pragma unroll
         for (int w = 0; w < kWarps; ++w)
             t += red[w];
+    }
+    __syncthreads();
+    return t;
+}
+
+// The same fixed-shape reduction for a CTA's sum of squares together with its
+// two range counters (results valid in thread 0; the binary64 sum is added in
+// the same order as block_sum's).
+struct CtaTotals {
+    double sq;
+    unsigned int nonzero, normal;
+};
+
+__device__ __forceinline__ CtaTotals block_totals(double x, unsigned int nz, unsigned int ns,
+                                                  double* red, uint2* ured)
+{
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1)
+        x += __shfl_down_sync(0xffffffffu, x, o);
+    nz = __reduce_add_sync(0xffffffffu, nz);
+    ns = __reduce_add_sync(0xffffffffu, ns);
+    if ((threadIdx.x & 31) == 0) {
+        red[threadIdx.x >> 5] = x;
+        ured[threadIdx.x >> 5] = make_uint2(nz, ns);
+    }
+    __syncthreads();
+    CtaTotals t{0.0, 0u, 0u};
+    if (threadIdx.x == 0) {
+#pragma unroll
+        for (int w = 0; w < kWarps; ++w) {
+            t.sq += red[w];
+            t.nonzero += ured[w].x;
+            t.normal += ured[w].y;
+        }
     }
     __syncthreads();
     return t;
@@ -541,6 +593,7 @@ __global__ void __launch_bounds__(kThreads, kStats == kMaxHist ? 4 : 8) check_ke
     __shared__ PackedStage st;
     __shared__ double s_red[kWarps];
     __shared__ unsigned int s_ured[kWarps];
+    __shared__ uint2 s_cnt[kWarps];
     __shared__ uint32_t s_hist[kStats == kMaxHist ? kThreads * kRow : 1];
     __shared__ int s_last;
 
@@ -569,6 +622,7 @@ __global__ void __launch_bounds__(kThreads, kStats == kMaxHist ? 4 : 8) check_ke
         q.pow2 = a.host_pow2 != 0;
     }
     SqAcc s;
+    RangeCounts rc;
     StatsAcc sa;
     if constexpr (kStats == kMaxHist) {
         sa.row = s_hist + threadIdx.x * kRow;
@@ -585,9 +639,9 @@ __global__ void __launch_bounds__(kThreads, kStats == kMaxHist ? 4 : 8) check_ke
         if (bin.kind == kChunkBin) {
             chunk_g = t.grads[bin.tensor] + bin.tensor_begin;
             if (q.pow2)
-                check_range<true, kStats>(chunk_g, bin.n_elems, q, s, &sa);
+                check_range<true, true, kStats>(chunk_g, bin.n_elems, q, s, &rc, &sa);
             else
-                check_range<false, kStats>(chunk_g, bin.n_elems, q, s, &sa);
+                check_range<false, true, kStats>(chunk_g, bin.n_elems, q, s, &rc, &sa);
         } else {
             stage_packed(bin, t, st);
             constexpr int kU = 8;
@@ -613,11 +667,12 @@ __global__ void __launch_bounds__(kThreads, kStats == kMaxHist ? 4 : 8) check_ke
                     for (int i = 0; i < kU; ++i)
                         sq_half<false>(h[i], q, s);
                 }
-                if constexpr (kStats != kNoStats) {
 #pragma unroll
-                    for (int i = 0; i < kU; ++i)
-                        if (in[i])
-                            stats_half<kStats>(h[i], &sa);
+                for (int i = 0; i < kU; ++i) {
+                    if (in[i]) {
+                        rc.half(h[i]);
+                        stats_half<kStats>(h[i], &sa);
+                    }
                 }
             }
         }
@@ -646,7 +701,8 @@ __global__ void __launch_bounds__(kThreads, kStats == kMaxHist ? 4 : 8) check_ke
         nf = block_sum_u32(c, s_ured);
     }
 
-    const double part = unscaled_sum(block_sum(s.a0 + s.a1, s_red), q);
+    const CtaTotals tot = block_totals(s.a0 + s.a1, rc.nonzero(), rc.normal(), s_red, s_cnt);
+    const double part = unscaled_sum(tot.sq, q);
     if constexpr (kStats != kNoStats) {
         const unsigned int mx = block_max_u32(sa.mx, s_ured);   // ends with __syncthreads
         if (kStats == kMaxHist && threadIdx.x < 32) {
@@ -664,8 +720,16 @@ __global__ void __launch_bounds__(kThreads, kStats == kMaxHist ? 4 : 8) check_ke
         a.partials[blockIdx.x] = part;
         if (nf)
             atomicAdd(&a.ctrl->nonfinite_acc, (unsigned long long)nf);
-        if (!valid)
+        if (valid) {
+            const unsigned int n_zero = (unsigned int)bin.n_elems - tot.nonzero;
+            const unsigned int n_sub = tot.nonzero - tot.normal;
+            if (n_zero)
+                atomicAdd(&a.ctrl->zero_acc, (unsigned long long)n_zero);
+            if (n_sub)
+                atomicAdd(&a.ctrl->subnormal_acc, (unsigned long long)n_sub);
+        } else {
             atomicOr(&a.ctrl->error_acc, (unsigned int)kErrBadBin);
+        }
     }
     // Two-level finish, so that the serial work after the last bin is small:
     // the last CTA to complete in each group of kFinishGroup consecutive bins
@@ -805,22 +869,6 @@ __device__ __forceinline__ void upd1(float g16f, float& w, float& v, const UpdPa
     w = __fsub_rn(w, s);
 }
 
-// Lane-packed counters: each 32-bit word carries two 16-bit counts (one per
-// FP16 lane); a thread adds at most 2^12 per lane, far below overflow.
-__device__ __forceinline__ void count_word(uint32_t w, uint32_t& nz2, uint32_t& ns2)
-{
-    const uint32_t m = w & 0x7FFF7FFFu;
-    nz2 += ((m + 0x7FFF7FFFu) >> 15) & 0x00010001u;  // lane != +-0
-    ns2 += ((m + 0x7C007C00u) >> 15) & 0x00010001u;  // lane >= 2^-14 (or inf/NaN)
-}
-
-__device__ __forceinline__ void count_half(uint16_t h, uint32_t& nz2, uint32_t& ns2)
-{
-    const uint32_t m = h & 0x7FFFu;
-    nz2 += m != 0 ? 1u : 0u;
-    ns2 += m >= 0x0400u ? 1u : 0u;
-}
-
 template <bool kStale>
 __device__ __forceinline__ void stale1(float w_old, float w_new, uint32_t& stale)
 {
@@ -831,8 +879,9 @@ __device__ __forceinline__ void stale1(float w_old, float w_new, uint32_t& stale
     }
 }
 
-// Four elements: 8-B FP16 gradient load, 16-B master and momentum loads,
-// 16-B + 16-B + 8-B stores (every warp access is 256 B or 512 B contiguous).
+// Four elements: the four FP16 gradients (two words), 16-B master and
+// momentum, 16-B + 16-B + 8-B stores (every warp access is 256 B or 512 B
+// contiguous).
 template <int kOpt, bool kStale>
 __device__ __forceinline__ void upd4(uint2 g, float4& w, float4& v, uint2& h, const UpdParams& p,
                                      uint32_t& stale)
@@ -865,201 +914,182 @@ __device__ __forceinline__ void upd_scalar(uint16_t g16, float* w, float* v, uin
     stale1<kStale>(w0, wi, stale);
 }
 
+// The four gradients of quad i (elements 4i .. 4i+3) of a range that starts
+// kS elements (2*kS bytes) past an 8-byte boundary, from the two aligned
+// 8-byte words that hold them: the upper 4 - kS elements of word i and the
+// lower kS of word i + 1 (word k holds elements 4k - kS .. 4k - kS + 3).
+template <int kS>
+__device__ __forceinline__ uint2 quad_from(uint2 lo, uint2 hi)
+{
+    uint2 q;
+    if constexpr (kS == 0) {
+        q = lo;
+    } else if constexpr (kS == 1) {
+        q.x = __funnelshift_r(lo.x, lo.y, 16);
+        q.y = __funnelshift_r(lo.y, hi.x, 16);
+    } else if constexpr (kS == 2) {
+        q.x = lo.y;
+        q.y = hi.x;
+    } else {
+        q.x = __funnelshift_r(lo.y, hi.x, 16);
+        q.y = __funnelshift_r(hi.x, hi.y, 16);
+    }
+    return q;
+}
+
+// Quads [i0, i1) of a range: master, momentum and FP16 copy are 16-/8-byte
+// aligned; the gradients start kS elements past an 8-byte boundary and are
+// read as aligned 8-byte words (two per quad when kS != 0, which the caller
+// keeps inside the range: i0 >= 1 and word i1 within it).  Each thread takes
+// quads i0 + threadIdx.x + k*kThreads, all four iterations' loads issued
+// before any is used (160 B in flight per thread).
+template <int kOpt, bool kStale, int kS>
+__device__ __forceinline__ void update_quads(const uint16_t* g, float* w, float* v, uint16_t* h,
+                                             int i0, int i1, const UpdParams& p, uint32_t& stale)
+{
+    constexpr int kUnroll = 4;
+    const uint2* gw = reinterpret_cast<const uint2*>(g - kS);
+    float4* w4 = reinterpret_cast<float4*>(w);
+    float4* v4 = reinterpret_cast<float4*>(v);
+    uint2* h4 = reinterpret_cast<uint2*>(h);
+    int i = i0 + (int)threadIdx.x;
+    for (; i + (kUnroll - 1) * kThreads < i1; i += kUnroll * kThreads) {
+        uint2 lo[kUnroll], hi[kUnroll], hq[kUnroll];
+        float4 wq[kUnroll], vq[kUnroll];
+#pragma unroll
+        for (int k = 0; k < kUnroll; ++k) {
+            lo[k] = __ldcs(gw + i + k * kThreads);
+            if constexpr (kS != 0)
+                hi[k] = __ldcs(gw + i + 1 + k * kThreads);
+            else
+                hi[k] = lo[k];
+            wq[k] = __ldcs(w4 + i + k * kThreads);
+            vq[k] = __ldcs(v4 + i + k * kThreads);
+        }
+#pragma unroll
+        for (int k = 0; k < kUnroll; ++k)
+            upd4<kOpt, kStale>(quad_from<kS>(lo[k], hi[k]), wq[k], vq[k], hq[k], p, stale);
+#pragma unroll
+        for (int k = 0; k < kUnroll; ++k) {
+            __stcs(w4 + i + k * kThreads, wq[k]);
+            __stcs(v4 + i + k * kThreads, vq[k]);
+            __stcs(h4 + i + k * kThreads, hq[k]);
+        }
+    }
+    for (; i < i1; i += kThreads) {
+        const uint2 lo = __ldcs(gw + i);
+        uint2 hi = lo;
+        if constexpr (kS != 0)
+            hi = __ldcs(gw + i + 1);
+        float4 wq = __ldcs(w4 + i), vq = __ldcs(v4 + i);
+        uint2 hq;
+        upd4<kOpt, kStale>(quad_from<kS>(lo, hi), wq, vq, hq, p, stale);
+        __stcs(w4 + i, wq);
+        __stcs(v4 + i, vq);
+        __stcs(h4 + i, hq);
+    }
+}
+
+// One contiguous range of a chunk bin at any 2-byte gradient alignment:
+// aligned quads with vector accesses; when the gradients are not 8-byte
+// aligned, the first quad and the elements past the last quad whose second
+// gradient word lies inside the range one element per thread.
 template <int kOpt, bool kStale>
 __device__ __forceinline__ void update_range(const uint16_t* g, float* w, float* v, uint16_t* h,
-                                             int len, const UpdParams& p, uint32_t& nz2,
-                                             uint32_t& ns2, uint32_t& stale)
+                                             int len, const UpdParams& p, uint32_t& stale)
 {
-    int start = 0;
-    if ((reinterpret_cast<uintptr_t>(g) & 7) == 0) {
-        constexpr int kUnroll = 4;
-        const uint2* g4 = reinterpret_cast<const uint2*>(g);
-        float4* w4 = reinterpret_cast<float4*>(w);
-        float4* v4 = reinterpret_cast<float4*>(v);
-        uint2* h4 = reinterpret_cast<uint2*>(h);
-        const int nq = len >> 2;
-        int i = threadIdx.x;
-        for (; i + (kUnroll - 1) * kThreads < nq; i += kUnroll * kThreads) {
-            uint2 gq[kUnroll], hq[kUnroll];
-            float4 wq[kUnroll], vq[kUnroll];
-#pragma unroll
-            for (int k = 0; k < kUnroll; ++k) {
-                gq[k] = __ldcs(g4 + i + k * kThreads);
-                wq[k] = __ldcs(w4 + i + k * kThreads);
-                vq[k] = __ldcs(v4 + i + k * kThreads);
-            }
-#pragma unroll
-            for (int k = 0; k < kUnroll; ++k) {
-                upd4<kOpt, kStale>(gq[k], wq[k], vq[k], hq[k], p, stale);
-                count_word(gq[k].x, nz2, ns2);
-                count_word(gq[k].y, nz2, ns2);
-            }
-#pragma unroll
-            for (int k = 0; k < kUnroll; ++k) {
-                __stcs(w4 + i + k * kThreads, wq[k]);
-                __stcs(v4 + i + k * kThreads, vq[k]);
-                __stcs(h4 + i + k * kThreads, hq[k]);
-            }
-        }
-        for (; i < nq; i += kThreads) {
-            uint2 gq = __ldcs(g4 + i), hq;
-            float4 wq = __ldcs(w4 + i), vq = __ldcs(v4 + i);
-            upd4<kOpt, kStale>(gq, wq, vq, hq, p, stale);
-            count_word(gq.x, nz2, ns2);
-            count_word(gq.y, nz2, ns2);
-            __stcs(w4 + i, wq);
-            __stcs(v4 + i, vq);
-            __stcs(h4 + i, hq);
-        }
-        start = nq << 2;
+    const int sh = (int)((reinterpret_cast<uintptr_t>(g) & 7u) >> 1);
+    int q1 = len >> 2;  // quads [q0, q1) go through the vector path
+    if (sh != 0) {
+        // quad i needs word i + 1, whose last element 4i + 7 - sh must be < len
+        q1 = len - 8 + sh >= 0 ? ((len - 8 + sh) >> 2) + 1 : 1;
+        if (q1 < 1)
+            q1 = 1;
     }
-    for (int j = start + threadIdx.x; j < len; j += kThreads) {
-        const uint16_t gh = __ldcs(g + j);
-        upd_scalar<kOpt, kStale>(gh, w + j, v + j, h + j, p, stale);
-        count_half(gh, nz2, ns2);
+    switch (sh) {
+    case 0: update_quads<kOpt, kStale, 0>(g, w, v, h, 0, q1, p, stale); break;
+    case 1: update_quads<kOpt, kStale, 1>(g, w, v, h, 1, q1, p, stale); break;
+    case 2: update_quads<kOpt, kStale, 2>(g, w, v, h, 1, q1, p, stale); break;
+    default: update_quads<kOpt, kStale, 3>(g, w, v, h, 1, q1, p, stale); break;
     }
+    if (sh != 0 && (int)threadIdx.x < min(4, len)) {
+        const int j = threadIdx.x;
+        upd_scalar<kOpt, kStale>(__ldcs(g + j), w + j, v + j, h + j, p, stale);
+    }
+    for (int j = 4 * q1 + (int)threadIdx.x; j < len; j += kThreads)
+        upd_scalar<kOpt, kStale>(__ldcs(g + j), w + j, v + j, h + j, p, stale);
 }
 
-// Overflow step: the update is skipped; only the range counts are taken.
-// Zero / subnormal counts of one contiguous range (16-B loads, four in
-// flight per thread, when the range is 16-B aligned).
-__device__ __forceinline__ void count_range(const uint16_t* g, int len, uint32_t& nz2, uint32_t& ns2)
-{
-    int start = 0;
-    if ((reinterpret_cast<uintptr_t>(g) & 15) == 0) {
-        constexpr int kU = 4;
-        const uint4* gv = reinterpret_cast<const uint4*>(g);
-        const int nv = len >> 3;
-        int i = threadIdx.x;
-        for (; i + (kU - 1) * kThreads < nv; i += kU * kThreads) {
-            uint4 q[kU];
-#pragma unroll
-            for (int k = 0; k < kU; ++k)
-                q[k] = __ldcs(gv + i + k * kThreads);
-#pragma unroll
-            for (int k = 0; k < kU; ++k) {
-                count_word(q[k].x, nz2, ns2);
-                count_word(q[k].y, nz2, ns2);
-                count_word(q[k].z, nz2, ns2);
-                count_word(q[k].w, nz2, ns2);
-            }
-        }
-        for (; i < nv; i += kThreads) {
-            const uint4 q = __ldcs(gv + i);
-            count_word(q.x, nz2, ns2);
-            count_word(q.y, nz2, ns2);
-            count_word(q.z, nz2, ns2);
-            count_word(q.w, nz2, ns2);
-        }
-        start = nv << 3;
-    }
-    for (int j = start + threadIdx.x; j < len; j += kThreads)
-        count_half(__ldcs(g + j), nz2, ns2);
-}
-
-// CTAs of an overflow step's update grid that take the range counts; the
-// rest exit at once.  592 = 4 CTAs (the update kernel's residency) per SM.
-constexpr int kCountCtas = 592;
-
-// Overflow step: nothing is updated, and the zero and subnormal counts are
-// taken by a sweep of the check pass's bins (64K-element ranges and the
-// packed bins): CTA k counts bins k, k + sweepers, ...  A bin's lane-packed
-// counts stay below 2^12 per lane (at most 2^20 elements per bin).
-template <bool kChecked>
-__device__ __forceinline__ void count_sweep(const Tables& t, const Bin* bins, int nbins,
-                                            int sweepers, Ctrl* ctrl, PackedStage& st,
-                                            unsigned int* s_ured)
-{
-    // t: segments, tensors and pointers (shared by both bin tables)
-    unsigned int n_el = 0, nz = 0, ns = 0;
-    bool bad = false;
-    for (int b = (int)blockIdx.x; b < nbins; b += sweepers) {
-        const Bin bin = bins[b];
-        if (kChecked && !bin_ok(bin, t)) {
-            bad = true;
-            continue;
-        }
-        uint32_t nz2 = 0, ns2 = 0;
-        if (bin.kind == kChunkBin) {
-            count_range(t.grads[bin.tensor] + bin.tensor_begin, bin.n_elems, nz2, ns2);
-        } else {
-            __syncthreads();  // nobody still reads the previous staging
-            stage_packed(bin, t, st);
-            for (int j = threadIdx.x; j < bin.n_elems; j += kThreads) {
-                const int k = find_seg(st.begin, bin.n_segs, j);
-                count_half(__ldcs(st.gptr[k] + (j - st.begin[k])), nz2, ns2);
-            }
-        }
-        nz += (nz2 & 0xFFFFu) + (nz2 >> 16);
-        ns += (ns2 & 0xFFFFu) + (ns2 >> 16);
-        n_el += (unsigned int)bin.n_elems;
-    }
-    const unsigned int bnz = block_sum_u32(nz, s_ured);
-    const unsigned int bns = block_sum_u32(ns, s_ured);
-    if (threadIdx.x == 0) {
-        atomicAdd(&ctrl->zero_acc, (unsigned long long)(n_el - bnz));
-        atomicAdd(&ctrl->subnormal_acc, (unsigned long long)(bnz - bns));
-        if (bad)
-            atomicOr(&ctrl->error, (unsigned int)kErrBadBin);
-    }
-}
-
+// Persistent grid: one CTA per resident slot (4 per SM; Adagrad 3).  CTA c
+// takes bin c first (counted from the end: the check kernel read the last
+// bins last, so their gradients are the ones still in L2) and then claims
+// further bins, gridDim.x + k for the k-th claim, from a counter that the
+// check kernel's last CTA resets every step.  An overflow step costs one
+// flag read per CTA.
 template <int kOpt, bool kStale, bool kChecked>
 __global__ void __launch_bounds__(kThreads, kOpt == kOptAdagrad ? 3 : 4) update_kernel(UpdateArgs a)
 {
     __shared__ PackedStage st;
+    __shared__ int s_next[2];
     __shared__ unsigned int s_ured[kWarps];
 
     const Tables& t = a.t;
-    // Bins run in reverse order: the check kernel read the last bins last, so
-    // their gradients are the ones still resident in L2.
-    const int b = t.nbins - 1 - (int)blockIdx.x;
-    const Bin bin = t.bins[b];
-    bool valid = true;
-    if constexpr (kChecked)
-        valid = bin_ok(bin, t);
-
-    // While the check kernel drains, start this CTA's first reads: a bulk
-    // (TMA) prefetch of the start of its master, momentum and gradient ranges
-    // into L2.  Whether to prefetch follows the overflow flag as the check
-    // kernel left it, read alongside the bin: this step's flag for a CTA that
-    // starts after the check has finished (most of the grid), the previous
-    // step's for one that starts while it drains.  It is only a hint: the
-    // update itself reads the flag after the wait.
-    if (valid && bin.kind == kChunkBin && threadIdx.x == 0 &&
-        *reinterpret_cast<const volatile int32_t*>(&a.ctrl->found_inf) == 0) {
-        const int n_pre = min(bin.n_elems, kPrefetchElems) & ~7;
-        if (n_pre > 0) {
-            prefetch_l2(a.master + bin.arena_begin, (uint32_t)n_pre * 4u);
-            prefetch_l2(a.momentum + bin.arena_begin, (uint32_t)n_pre * 4u);
-            const uint16_t* g = t.grads[bin.tensor] + bin.tensor_begin;
-            if ((reinterpret_cast<uintptr_t>(g) & 15) == 0)
-                prefetch_l2(g, (uint32_t)n_pre * 2u);
+    const int nb = t.nbins;
+    int idx = (int)blockIdx.x;
+    if (idx >= nb)
+        return;
+    {
+        // While the check kernel drains, start this CTA's first reads: a
+        // bulk (TMA) prefetch of the start of its first bin's master,
+        // momentum and gradient ranges into L2.  Whether to prefetch follows
+        // the overflow flag as the check kernel left it: this step's flag
+        // for a CTA that starts after the check has finished, the previous
+        // step's for one that starts while it drains.  It is only a hint:
+        // the update itself reads the flag after the wait.
+        const Bin bin = t.bins[nb - 1 - idx];
+        bool ok = true;
+        if constexpr (kChecked)
+            ok = bin_ok(bin, t);
+        if (ok && bin.kind == kChunkBin && threadIdx.x == 0 &&
+            *reinterpret_cast<const volatile int32_t*>(&a.ctrl->found_inf) == 0) {
+            const int n_pre = min(bin.n_elems, kPrefetchElems) & ~7;
+            if (n_pre > 0) {
+                prefetch_l2(a.master + bin.arena_begin, (uint32_t)n_pre * 4u);
+                prefetch_l2(a.momentum + bin.arena_begin, (uint32_t)n_pre * 4u);
+                const uint16_t* g = t.grads[bin.tensor] + bin.tensor_begin;
+                if ((reinterpret_cast<uintptr_t>(g) & 15) == 0)
+                    prefetch_l2(g, (uint32_t)n_pre * 2u);
+            }
         }
     }
     // Wait until the check kernel has finished and its result is visible
     // (returns at once when this grid was launched without overlap).
     asm volatile("griddepcontrol.wait;" ::: "memory");
-    const Ctrl* c = a.ctrl;
+    Ctrl* c = a.ctrl;
     if (c->found_inf != 0) {
         // Overflow step (Step 6): master, momentum and FP16 copy stay as they
-        // are.  The flag is the same for every thread of the grid, so the
-        // branch is uniform.  (Checked mode: the sweep validates the check
-        // bins it walks; this grid's own bins are validated on the next step
-        // that uses them.)
-        const int sweepers = min(kCountCtas, (int)gridDim.x);
-        if ((int)blockIdx.x < sweepers)
-            count_sweep<kChecked>(t, a.check_bins, a.check_nbins, sweepers, a.ctrl, st, s_ured);
+        // are.  The flag is the same for every thread of the grid.
         return;
     }
     const UpdParams p{c->inv_scale, c->coef, a.lr, a.mu, a.wd, a.eps};
-    uint32_t nz2 = 0, ns2 = 0, stale = 0;
+    uint32_t stale = 0;
+    bool bad = false;
 
-    if (valid) {
-        if (bin.kind == kChunkBin) {
+    for (int it = 0; idx < nb; ++it) {
+        // claim the next bin now; its number is needed only after this one
+        unsigned int claim = 0;
+        if (threadIdx.x == 0)
+            claim = atomicAdd(&c->upd_next, 1u);
+        const Bin bin = t.bins[nb - 1 - idx];
+        bool valid = true;
+        if constexpr (kChecked)
+            valid = bin_ok(bin, t);
+        if (!valid) {
+            bad = true;
+        } else if (bin.kind == kChunkBin) {
             const uint16_t* g = t.grads[bin.tensor] + bin.tensor_begin;
             update_range<kOpt, kStale>(g, a.master + bin.arena_begin, a.momentum + bin.arena_begin,
-                                       a.w16 + bin.arena_begin, bin.n_elems, p, nz2, ns2, stale);
+                                       a.w16 + bin.arena_begin, bin.n_elems, p, stale);
         } else {
             stage_packed(bin, t, st);
             constexpr int kU = 4;
@@ -1084,7 +1114,6 @@ __global__ void __launch_bounds__(kThreads, kOpt == kOptAdagrad ? 3 : 4) update_
                 for (int i = 0; i < kU; ++i) {
                     if (e[i] < 0)
                         continue;
-                    count_half(gh[i], nz2, ns2);
                     const float w0 = w[i];
                     upd1<kOpt>(__half2float(__ushort_as_half(gh[i])), w[i], v[i], p);
                     __stcs(a.master + e[i], w[i]);
@@ -1094,24 +1123,21 @@ __global__ void __launch_bounds__(kThreads, kOpt == kOptAdagrad ? 3 : 4) update_
                 }
             }
         }
+        // the next bin's number; the barrier also ends every read of the
+        // packed staging before the next bin may overwrite it
+        if (threadIdx.x == 0)
+            s_next[it & 1] = (int)gridDim.x + (int)claim;
+        __syncthreads();
+        idx = s_next[it & 1];
     }
 
-    const unsigned int nz = block_sum_u32((nz2 & 0xFFFFu) + (nz2 >> 16), s_ured);
-    const unsigned int ns = block_sum_u32((ns2 & 0xFFFFu) + (ns2 >> 16), s_ured);
-    unsigned int n_stale = 0;
-    if constexpr (kStale)
-        n_stale = block_sum_u32(stale, s_ured);
-    if (threadIdx.x == 0) {
-        Ctrl* cw = a.ctrl;
-        if (valid) {
-            atomicAdd(&cw->zero_acc, (unsigned long long)(bin.n_elems - nz));
-            atomicAdd(&cw->subnormal_acc, (unsigned long long)(nz - ns));
-            if (n_stale)
-                atomicAdd(&cw->stale_acc, (unsigned long long)n_stale);
-        } else {
-            atomicOr(&cw->error, (unsigned int)kErrBadBin);
-        }
+    if constexpr (kStale) {
+        const unsigned int n_stale = block_sum_u32(stale, s_ured);
+        if (threadIdx.x == 0 && n_stale)
+            atomicAdd(&c->stale_acc, (unsigned long long)n_stale);
     }
+    if (kChecked && bad && threadIdx.x == 0)
+        atomicOr(&c->error, (unsigned int)kErrBadBin);
 }
 
 // ---------------------------------------------------------------------------

@@ -67,18 +67,28 @@ class ShardedMPT:
     def device_scale(self):
         return self.opt.device_scale()
 
-    def step(self, flat_grads, lr, momentum, weight_decay, clip=0.0):
+    def step(self, flat_grads, lr, momentum, weight_decay, clip=0.0, marks=None):
         """``flat_grads``: this rank's FP16 gradients of the whole list, padded
         to ``padded`` elements (zeros past ``total``).  Returns the full FP16
-        weights (a view of ``total`` elements)."""
+        weights (a view of ``total`` elements).  ``marks``: optional list of
+        six CUDA timing events, recorded on the current stream before the
+        reduce-scatter and after each of the five phases (reduce-scatter,
+        check pass, record all-gather, finish and update, FP16 all-gather)."""
         if flat_grads.numel() != self.padded or flat_grads.element_size() != 2:
             raise ValueError(f"expected {self.padded} FP16 gradients")
+        mark = (lambda i: marks[i].record()) if marks is not None else (lambda i: None)
+        mark(0)
         dist.reduce_scatter_tensor(self.grad_shard, flat_grads, op=dist.ReduceOp.SUM,
                                    group=self.group)
+        mark(1)
         mine = self.opt.step_partial([self.grad_shard])
+        mark(2)
         exchange_records(self.records, mine, self.group)
+        mark(3)
         self.opt.step_finish(self.records, self.world, lr, momentum, weight_decay, clip)
+        mark(4)
         dist.all_gather_into_tensor(self.w16_full, self.opt.w16(0), group=self.group)
+        mark(5)
         return self.w16_full[: self.total]
 
     def wait(self):

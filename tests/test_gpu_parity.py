@@ -99,8 +99,11 @@ def test_edge_sizes(sizes):
 
 @pytest.mark.parametrize("shift", [0, 1, 2, 3, 4, 5, 6, 7])
 def test_unaligned_gradient_pointers(shift):
-    # 2-, 4-, 6-, 8-, ... byte offsets select the 16-B, 8-B and 2-B load paths
-    cfg = custom([10_000, 70_001, 33], steps=2)
+    # 2-, 4-, 6-, 8-, ... byte offsets: the check pass's per-thread head
+    # before the first 16-byte boundary, the update's shifted gradient words
+    # (0-3 elements past an 8-byte boundary) and its scalar first quad and
+    # tail; update bins of 1025 elements and tails of 1, 5, 7 and 8 elements
+    cfg = custom([10_000, 70_001, 33, 1025, 4097, 4101, 4103, 4104, 4105], steps=2)
     p = Pair(cfg)
     for step in (1, 2):
         host = p.grads(step, p.scale)
@@ -377,6 +380,35 @@ def test_async_steps_follow_the_oracle():
     st = p.opt.stats()
     assert st["steps"] == cfg.steps and st["skipped"] == 2
     p.compare_state("after queued steps", exact=True)
+
+
+def test_stale_total_over_queued_steps():
+    """With MPT_FLAG_COUNT_STALE, the running total of stale FP16 elements
+    (master moved, rounded copy did not) must count every step queued between
+    two waits, not only the last one; an overflow step adds nothing."""
+    plan = {3: [(0, 11, 0x7C00)]}
+    cfg = custom([60_000, 1031, 5, 40_000], law=("log2_uniform", -26.0, -6.0), scale0=2.0 ** 12,
+                 growth_interval=0, lr=1e-3, steps=6, injections=lambda s: plan.get(s, []))
+    p = Pair(cfg, flags=MPT_FLAG_COUNT_STALE)
+    S, per_step, bufs = cfg.scale0, [], []
+    for k in range(1, 6):
+        host = p.grads(k, S)
+        dev = host.cuda()
+        bufs.append(dev)
+        p.opt.step_async(p.layout.views(dev), cfg.lr, cfg.momentum, cfg.weight_decay)
+        hv = [v.numpy().view(np.uint16) for v in p.layout.views(host)]
+        ro = oracle.step(p.state, hv, S, cfg.lr, cfg.momentum, cfg.weight_decay, cfg=p.ocfg)
+        per_step.append(ro["n_stale"])
+        S = ro["new_scale"]
+    r = p.opt.wait()
+    assert per_step[2] == 0 and min(per_step[:2] + per_step[3:]) > 0
+    assert r["n_fp16_stale"] == per_step[-1]
+    assert p.opt.stats()["n_fp16_stale_total"] == sum(per_step)
+    # a waiting step after the queued ones adds its own count
+    r2, ro2 = p.step()
+    assert r2["n_fp16_stale"] == ro2["n_stale"]
+    assert p.opt.stats()["n_fp16_stale_total"] == sum(per_step) + ro2["n_stale"]
+    p.compare_state("after queued stale steps", exact=True)
 
 
 def test_sync_and_async_steps_share_the_scale_state():
