@@ -124,7 +124,8 @@ typedef struct {
     float clip_coef;       /* clip / grad_norm when clipped, else 1             */
     float max_abs_grad;    /* MPT_FLAG_GRAD_STATS / direct mode, else 0: the
                               largest unscaled finite |g|, fp32(max|g16|)*(1/S) */
-    uint64_t n_zero;       /* FP16 gradients equal to +-0                       */
+    uint64_t n_zero;       /* FP16 gradients equal to +-0 (counted by the check
+                              pass, so overflow steps report them too)         */
     uint64_t n_subnormal;  /* FP16 gradients with 0 < |g16| < 2^-14             */
     uint64_t n_nonfinite;  /* FP16 gradients that are +-inf or NaN              */
     uint64_t n_fp16_stale; /* MPT_FLAG_COUNT_STALE only, else 0: elements whose
@@ -137,7 +138,9 @@ typedef struct {
     float scale;              /* current S (last new_scale, or the value set)   */
     int32_t clean_run;        /* current clean-step counter                     */
     mpt_step_result last;     /* result of the last completed step              */
-    uint64_t n_fp16_stale_total;
+    uint64_t n_fp16_stale_total; /* MPT_FLAG_COUNT_STALE: n_fp16_stale summed
+                              over every step since creation, queued ones
+                              included (summed on the device)                 */
     uint64_t timed_steps;     /* steps timed while mpt_set_timing was on        */
     double check_ms_total;    /* summed CUDA-event durations of the check       */
     double update_ms_total;   /* kernel and of the update kernel over them      */
@@ -355,12 +358,18 @@ const char* mpt_error_string(int code);
  *                 mpt_check_result when the queued work completes
  *   cuda_stream   stream to queue on; the call returns without waiting
  *
- * The first call on each device looks up the device address of the scratch
- * array (with that device current); make that first call before any stream
- * capture.  Every call on a device shares the one scratch array, which keeps
- * the last call's contents; each call clears the counters it needs before its
- * kernel runs.  Calls whose work overlaps on the GPU (other streams, other
- * host threads) race on that array and give wrong results: serialize them.
+ * The first successful call on each device sets that device up, with it
+ * current: it looks up the device address of the scratch array and loads the
+ * call's kernels (both of its variants, for power-of-two and other S), so no
+ * later call loads code.  Make that first call before any stream capture; a
+ * set-up that fails (inside a capture, say) returns MPT_ERR_CUDA, keeps
+ * nothing, and the next call tries again.  Every call on a device shares the
+ * one scratch array, which keeps the last call's contents; each call clears
+ * the counters it needs before its kernel runs.  Calls whose work overlaps on
+ * the GPU (other streams, other host threads) race on that array and give
+ * wrong results: serialize them.  The call checks the status each CUDA call
+ * returns; it clears the runtime's last-error state only after a failure of
+ * its own, so an error left pending by earlier work stays for the caller.
  * Errors: MPT_ERR_INVALID_ARG, MPT_ERR_TOO_LARGE, MPT_ERR_CUDA. */
 #define MPT_NOALLOC_MAX_ELEMS (((int64_t)1) << 30)
 

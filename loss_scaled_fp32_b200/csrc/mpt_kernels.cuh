@@ -731,40 +731,56 @@ __global__ void __launch_bounds__(kThreads, kStats == kMaxHist ? 4 : 8) check_ke
             atomicOr(&a.ctrl->error_acc, (unsigned int)kErrBadBin);
         }
     }
-    // Two-level finish, so that the serial work after the last bin is small:
-    // the last CTA to complete in each group of kFinishGroup consecutive bins
-    // adds that group's partials (in bin order, fixed pattern); the last
-    // group to complete adds the group sums (in group order) and finishes the
-    // step.  Fences before each ticket make every counter and partial written
-    // before it visible to the CTA that draws the last ticket.
+    // Finish by atomic tickets (the last CTA to draw one sees every partial
+    // and counter: fences before each ticket make them visible).  Up to
+    // kOneLevelBins bins, one level: the last CTA adds all the partials (at
+    // most eight loads per thread, issued together).  Beyond, two levels, so
+    // that the serial work after the last bin stays small: the last CTA to
+    // complete in each group of kFinishGroup consecutive bins adds that
+    // group's partials; the last group to complete adds the group sums.
+    // Either way the additions follow a fixed pattern (bin order within a
+    // thread's share, a fixed tree across threads), whichever CTA is last.
     __syncthreads();  // every write of this CTA precedes its ticket
-    const int grp = (int)blockIdx.x / kFinishGroup;
-    const int g_begin = grp * kFinishGroup;
-    const int g_len = min(kFinishGroup, (int)gridDim.x - g_begin);
-    if (threadIdx.x == 0) {
+    double sumsq;
+    if ((int)gridDim.x <= kOneLevelBins) {
+        if (threadIdx.x == 0) {
+            __threadfence();
+            s_last = atomicAdd(&a.ctrl->ticket, 1u) == gridDim.x - 1;
+        }
+        __syncthreads();
+        if (!s_last)
+            return;
         __threadfence();
-        s_last = atomicAdd(&a.group_tickets[grp], 1u) == (unsigned int)g_len - 1;
-    }
-    __syncthreads();
-    if (!s_last)
-        return;
-    __threadfence();
-    const double gsum = block_sum(
-        threadIdx.x < g_len ? __ldcg(a.partials + g_begin + threadIdx.x) : 0.0, s_red);
-    const int ngroups = ((int)gridDim.x + kFinishGroup - 1) / kFinishGroup;
-    if (threadIdx.x == 0) {
-        a.group_partials[grp] = gsum;
-        a.group_tickets[grp] = 0;
+        sumsq = block_sum(sum_partials(a.partials, (int)gridDim.x), s_red);
+    } else {
+        const int grp = (int)blockIdx.x / kFinishGroup;
+        const int g_begin = grp * kFinishGroup;
+        const int g_len = min(kFinishGroup, (int)gridDim.x - g_begin);
+        if (threadIdx.x == 0) {
+            __threadfence();
+            s_last = atomicAdd(&a.group_tickets[grp], 1u) == (unsigned int)g_len - 1;
+        }
+        __syncthreads();
+        if (!s_last)
+            return;
         __threadfence();
-        s_last = atomicAdd(&a.ctrl->ticket, 1u) == (unsigned int)ngroups - 1;
+        const double gsum = block_sum(
+            threadIdx.x < g_len ? __ldcg(a.partials + g_begin + threadIdx.x) : 0.0, s_red);
+        const int ngroups = ((int)gridDim.x + kFinishGroup - 1) / kFinishGroup;
+        if (threadIdx.x == 0) {
+            a.group_partials[grp] = gsum;
+            a.group_tickets[grp] = 0;
+            __threadfence();
+            s_last = atomicAdd(&a.ctrl->ticket, 1u) == (unsigned int)ngroups - 1;
+        }
+        __syncthreads();
+        if (!s_last)
+            return;
+        __threadfence();
+        sumsq = block_sum(sum_partials(a.group_partials, ngroups), s_red);
     }
-    __syncthreads();
-    if (!s_last)
-        return;
 
-    // Last group: every CTA's partial and counters are visible.
-    __threadfence();
-    const double sumsq = block_sum(sum_partials(a.group_partials, ngroups), s_red);
+    // Last CTA: every CTA's partial and counters are visible.
     Ctrl* c = a.ctrl;
     if constexpr (kStats == kMaxHist) {
         if (threadIdx.x < 32) {
