@@ -263,9 +263,18 @@ __device__ __forceinline__ double sq_value(float g, const SqParams& a)
 template <bool kPow2>
 __device__ __forceinline__ void sq_word(uint32_t w, const SqParams& a, SqAcc& s)
 {
-    const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&w));
-    const double x0 = sq_value<kPow2>(f.x, a);
-    const double x1 = sq_value<kPow2>(f.y, a);
+    double x0, x1;
+    if constexpr (kPow2) {
+        // the two binary16 lanes widened straight to binary64 (exact): one
+        // conversion per gradient instead of two
+        asm("{\n\t.reg .f16 lo, hi;\n\tmov.b32 {lo, hi}, %2;\n\t"
+            "cvt.f64.f16 %0, lo;\n\tcvt.f64.f16 %1, hi;\n\t}"
+            : "=d"(x0), "=d"(x1) : "r"(w));
+    } else {
+        const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&w));
+        x0 = sq_value<kPow2>(f.x, a);
+        x1 = sq_value<kPow2>(f.y, a);
+    }
     s.a0 = fma(x0, x0, s.a0);
     s.a1 = fma(x1, x1, s.a1);
 }
@@ -340,19 +349,39 @@ __device__ __forceinline__ void stats_vec(uint4 v, StatsAcc* st)
 
 // Range counts of the gradients (how many are +-0 and how many are
 // subnormal in binary16: the part of the gradient distribution that FP16
-// flushes or keeps only with reduced precision).  Lane-packed counters: each
-// 32-bit word carries two 16-bit counts, one per FP16 lane of a gradient
-// word; a thread adds at most 2^11 per lane (at most 2^20 elements per bin),
-// far below overflow.
+// flushes or keeps only with reduced precision).
+//
+// Per gradient word (two binary16 lanes), with m = the lanes' magnitudes:
+// m + 0x7FFF sets a lane's bit 15 iff the lane is not +-0, m + 0x7C00 iff it
+// is at least 2^-14 (normal, inf or NaN).  One byte permute gathers the four
+// flag bytes into byte lanes [nonzero lo, nonzero hi, normal lo, normal hi]
+// that accumulate in b4 (at most 16 per byte between two folds: one batch of
+// kCheckVecs 16-byte vectors); fold() moves them into lane-packed 16-bit
+// counters, of which a thread fills at most 2^11 per lane (at most 2^20
+// elements per bin), far below overflow.
 struct RangeCounts {
     uint32_t nz2 = 0;  // lanes with |g16| != 0
     uint32_t ns2 = 0;  // lanes with |g16| >= 2^-14 (normal, inf or NaN)
+    uint32_t b4 = 0;   // byte lanes, see above
 
     __device__ __forceinline__ void word(uint32_t w)
     {
         const uint32_t m = w & 0x7FFF7FFFu;
-        nz2 += ((m + 0x7FFF7FFFu) >> 15) & 0x00010001u;  // lane != +-0
-        ns2 += ((m + 0x7C007C00u) >> 15) & 0x00010001u;  // lane >= 2^-14
+        const uint32_t p = __byte_perm(m + 0x7FFF7FFFu, m + 0x7C007C00u, 0x7531);
+        b4 += (p >> 7) & 0x01010101u;
+    }
+    __device__ __forceinline__ void vec(uint4 v)
+    {
+        word(v.x);
+        word(v.y);
+        word(v.z);
+        word(v.w);
+    }
+    __device__ __forceinline__ void fold()
+    {
+        nz2 += __byte_perm(b4, 0, 0x4140);  // bytes 0, 1 -> the two 16-bit lanes
+        ns2 += __byte_perm(b4, 0, 0x4342);  // bytes 2, 3
+        b4 = 0;
     }
     __device__ __forceinline__ void half(uint16_t h)
     {
@@ -395,23 +424,19 @@ __device__ __forceinline__ void check_range_vec(const uint16_t* g, int len, cons
 #pragma unroll
         for (int k = 0; k < kU; ++k) {
             sq_vec<kPow2>(v[k], a, s);
-            if constexpr (kCount) {
-                rc->word(v[k].x);
-                rc->word(v[k].y);
-                rc->word(v[k].z);
-                rc->word(v[k].w);
-            }
+            if constexpr (kCount)
+                rc->vec(v[k]);
             stats_vec<kStats>(v[k], st);
         }
+        if constexpr (kCount)
+            rc->fold();
     }
     for (; i < nv; i += kThreads) {
         const uint4 v = __ldg(gv + i);
         sq_vec<kPow2>(v, a, s);
         if constexpr (kCount) {
-            rc->word(v.x);
-            rc->word(v.y);
-            rc->word(v.z);
-            rc->word(v.w);
+            rc->vec(v);
+            rc->fold();
         }
         stats_vec<kStats>(v, st);
     }
@@ -1038,10 +1063,11 @@ __device__ __forceinline__ void update_range(const uint16_t* g, float* w, float*
 
 // Persistent grid: one CTA per resident slot (4 per SM; Adagrad 3).  CTA c
 // takes bin c first (counted from the end: the check kernel read the last
-// bins last, so their gradients are the ones still in L2) and then claims
-// further bins, gridDim.x + k for the k-th claim, from a counter that the
-// check kernel's last CTA resets every step.  An overflow step costs one
-// flag read per CTA.
+// bins last, so their gradients are the ones still in L2) and then, each time
+// it finishes a bin, claims the next one, gridDim.x + k for the k-th claim,
+// from a counter that the check kernel's last CTA resets every step: bins
+// start in order, and an SM that streams faster takes more of them.  An
+// overflow step costs one flag read per CTA.
 template <int kOpt, bool kStale, bool kChecked>
 __global__ void __launch_bounds__(kThreads, kOpt == kOptAdagrad ? 3 : 4) update_kernel(UpdateArgs a)
 {
@@ -1081,21 +1107,19 @@ __global__ void __launch_bounds__(kThreads, kOpt == kOptAdagrad ? 3 : 4) update_
     // Wait until the check kernel has finished and its result is visible
     // (returns at once when this grid was launched without overlap).
     asm volatile("griddepcontrol.wait;" ::: "memory");
+    // the check result, read past L1 (the hint above may have cached the
+    // line before the check kernel's last CTA wrote it)
     Ctrl* c = a.ctrl;
-    if (c->found_inf != 0) {
+    if (__ldcg(&c->found_inf) != 0) {
         // Overflow step (Step 6): master, momentum and FP16 copy stay as they
         // are.  The flag is the same for every thread of the grid.
         return;
     }
-    const UpdParams p{c->inv_scale, c->coef, a.lr, a.mu, a.wd, a.eps};
+    const UpdParams p{__ldcg(&c->inv_scale), __ldcg(&c->coef), a.lr, a.mu, a.wd, a.eps};
     uint32_t stale = 0;
     bool bad = false;
 
     for (int it = 0; idx < nb; ++it) {
-        // claim the next bin now; its number is needed only after this one
-        unsigned int claim = 0;
-        if (threadIdx.x == 0)
-            claim = atomicAdd(&c->upd_next, 1u);
         const Bin bin = t.bins[nb - 1 - idx];
         bool valid = true;
         if constexpr (kChecked)
@@ -1139,10 +1163,12 @@ __global__ void __launch_bounds__(kThreads, kOpt == kOptAdagrad ? 3 : 4) update_
                 }
             }
         }
-        // the next bin's number; the barrier also ends every read of the
-        // packed staging before the next bin may overwrite it
+        // claim the next bin once this one is done (claiming earlier holds a
+        // bin back from CTAs that free up sooner and lengthens the tail);
+        // the barrier also ends every read of the packed staging before the
+        // next bin may overwrite it
         if (threadIdx.x == 0)
-            s_next[it & 1] = (int)gridDim.x + (int)claim;
+            s_next[it & 1] = (int)gridDim.x + (int)atomicAdd(&c->upd_next, 1u);
         __syncthreads();
         idx = s_next[it & 1];
     }
