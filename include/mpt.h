@@ -212,14 +212,22 @@ int mpt_step(mpt_handle* h, const void* const* d_grads_half, float scale,
  * state on the device.  Nothing is read back; call mpt_wait for the result
  * of the last queued step.  The gradient buffers must stay unchanged until
  * the queued work has run.
- * CUDA graphs: when d_grads_half holds the same pointers as the previous
- * step of this handle, the call queues exactly the two kernel launches (no
- * copy, no host synchronisation), so it can be captured into a CUDA graph
- * (kernel timing off).  Each replay reads the gradients its buffers hold at
- * replay time and reads and advances the device scale state; mpt_wait on
- * the replay stream returns the replayed step's result.  With new pointers
- * the call first copies the pointer table from pinned host memory, which a
- * capture must not record.
+ * Gradient-pointer tables: the handle keeps device copies of the last four
+ * distinct tables passed to its steps (in its workspace).  A step whose
+ * d_grads_half equals one of them queues exactly the two kernel launches (no
+ * copy, no host synchronisation); a new table is copied from pinned host
+ * memory into the least recently used copy first, ordered on the step's
+ * stream after the steps queued before it.  So queue a handle's steps on one
+ * stream (or order its streams yourself).
+ * CUDA graphs: a step whose table is already held queues only the two
+ * kernel launches, so it can be captured into a CUDA graph (kernel timing
+ * off); capture only after a first, uncaptured step with the same table (a
+ * new table's copy must not be recorded).  Each replay reads the gradients
+ * its buffers hold at replay time, the pointer copy that the capture used,
+ * and reads and advances the device scale state; mpt_wait on the replay
+ * stream returns the replayed step's result.  A later step with a fifth
+ * distinct table may rewrite that copy: replay a captured step only while
+ * its table is among the last four used.
  * Errors: MPT_ERR_INVALID_ARG, MPT_ERR_CUDA, MPT_ERR_BROKEN. */
 int mpt_step_async(mpt_handle* h, const void* const* d_grads_half, float lr,
                    float momentum, float weight_decay, float clip, void* cuda_stream);

@@ -38,6 +38,10 @@ static_assert(offsetof(Ctrl, stale_acc) == 128 && offsetof(Ctrl, sumsq) == 256,
 namespace {
 
 constexpr size_t kRegionAlign = 256;
+// Device copies of the caller's gradient-pointer table kept at once: a step
+// whose pointers match one of them queues no copy (a training loop that
+// alternates a few gradient buffers switches between cached tables).
+constexpr int kPtrSlots = 4;
 
 size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
@@ -185,7 +189,7 @@ int build_layout(const int64_t* sizes, int32_t n, int32_t check_chunk, int32_t u
     const size_t ngroups = (L.bins_check.size() + kFinishGroup - 1) / kFinishGroup;
     L.off_groups = region(sizeof(double) * ngroups);
     L.off_group_tickets = region(sizeof(unsigned int) * ngroups);
-    L.off_ptrs = region(sizeof(void*) * (size_t)n);
+    L.off_ptrs = region(sizeof(void*) * (size_t)n * kPtrSlots);
     L.off_tinfo = region(sizeof(TensorInfo) * (size_t)n);
     L.off_bins_check = region(sizeof(Bin) * L.bins_check.size());
     L.off_bins_update = region(sizeof(Bin) * L.bins_update.size());
@@ -247,10 +251,19 @@ struct mpt_handle {
     uint16_t* d_w16 = nullptr;
     int32_t upd_grid = 0;                // CTAs of the persistent update grid
     // host state
-    std::vector<const void*> last_ptrs;
-    bool ptrs_uploaded = false;
-    const void** pinned_ptrs = nullptr;  // staging of the pointer table
-    cudaEvent_t ptrs_copied = nullptr;   // the last pointer-table copy is done
+    // gradient-pointer tables: slot k holds a device copy (d_ptrs + k*n) of
+    // the host table ptrs, staged through pinned; copied marks the end of its
+    // last copy; used orders the slots by last use
+    struct PtrSlot {
+        std::vector<const void*> ptrs;
+        bool valid = false;
+        uint64_t used = 0;
+        const void** pinned = nullptr;
+        cudaEvent_t copied = nullptr;
+    };
+    PtrSlot slot[kPtrSlots];
+    int cur_slot = -1;                   // the slot of the last step (-1: none)
+    uint64_t slot_clock = 0;
     Ctrl* mailbox = nullptr;             // pinned copy of the control block
     unsigned long long* hist_box = nullptr;  // pinned copy of the histogram
     uint64_t hist[32] = {};
@@ -274,10 +287,12 @@ static void release(mpt_handle* h)
     for (cudaEvent_t e : h->tev)
         if (e)
             cudaEventDestroy(e);
-    if (h->ptrs_copied)
-        cudaEventDestroy(h->ptrs_copied);
-    if (h->pinned_ptrs)
-        cudaFreeHost(h->pinned_ptrs);
+    for (auto& sl : h->slot) {
+        if (sl.copied)
+            cudaEventDestroy(sl.copied);
+        if (sl.pinned)
+            cudaFreeHost(sl.pinned);
+    }
     if (h->mailbox)
         cudaFreeHost(h->mailbox);
     if (h->hist_box)
@@ -451,7 +466,7 @@ static int enqueue_step(mpt_handle* h, const void* const* d_grads_half, bool sca
     NvtxRange range(phase == Phase::kWhole ? "mpt.step" :
                     phase == Phase::kShardCheck ? "mpt.step_partial" : "mpt.step_finish");
     if (phase == Phase::kShardFinish)
-        d_grads_half = h->last_ptrs.data();  // the pointers of the check pass
+        d_grads_half = h->slot[h->cur_slot].ptrs.data();  // the pointers of the check pass
     for (int32_t i = 0; i < h->n; ++i) {
         const uintptr_t p = reinterpret_cast<uintptr_t>(d_grads_half[i]);
         if (p == 0 || (p & 1))
@@ -464,24 +479,40 @@ static int enqueue_step(mpt_handle* h, const void* const* d_grads_half, bool sca
     }
     const size_t ptr_bytes = sizeof(void*) * (size_t)h->n;
 
-    // The pointer table crosses to the device only when it changed; the
-    // staging buffer is reused only once its previous copy has completed.
-    if (!h->ptrs_uploaded || std::memcmp(h->last_ptrs.data(), d_grads_half, ptr_bytes) != 0) {
-        if (h->ptrs_uploaded && cudaEventSynchronize(h->ptrs_copied) != cudaSuccess)
+    // The pointer table crosses to the device only when no cached slot holds
+    // it: then the least recently used slot is rewritten (stream-ordered
+    // after the steps queued before that read it; its staging buffer is
+    // reused only once its previous copy has completed).
+    int k = -1;
+    if (h->cur_slot >= 0 && std::memcmp(h->slot[h->cur_slot].ptrs.data(), d_grads_half, ptr_bytes) == 0)
+        k = h->cur_slot;
+    for (int i = 0; k < 0 && i < kPtrSlots; ++i)
+        if (h->slot[i].valid && std::memcmp(h->slot[i].ptrs.data(), d_grads_half, ptr_bytes) == 0)
+            k = i;
+    if (k < 0) {
+        k = 0;
+        for (int i = 1; i < kPtrSlots; ++i)
+            if (!h->slot[i].valid ? h->slot[k].valid : (h->slot[k].valid && h->slot[i].used < h->slot[k].used))
+                k = i;
+        auto& sl = h->slot[k];
+        if (sl.valid && cudaEventSynchronize(sl.copied) != cudaSuccess)
             return MPT_ERR_CUDA;
-        std::memcpy(h->pinned_ptrs, d_grads_half, ptr_bytes);
-        if (cudaMemcpyAsync(h->d_ptrs, h->pinned_ptrs, ptr_bytes, cudaMemcpyHostToDevice, st) != cudaSuccess ||
-            cudaEventRecord(h->ptrs_copied, st) != cudaSuccess)
+        sl.valid = false;
+        std::memcpy(sl.pinned, d_grads_half, ptr_bytes);
+        if (cudaMemcpyAsync(h->d_ptrs + (size_t)k * h->n, sl.pinned, ptr_bytes, cudaMemcpyHostToDevice, st) != cudaSuccess ||
+            cudaEventRecord(sl.copied, st) != cudaSuccess)
             return MPT_ERR_CUDA;
-        std::memcpy(h->last_ptrs.data(), d_grads_half, ptr_bytes);
-        h->ptrs_uploaded = true;
+        std::memcpy(sl.ptrs.data(), d_grads_half, ptr_bytes);
+        sl.valid = true;
     }
+    h->slot[k].used = ++h->slot_clock;
+    h->cur_slot = k;
 
     Tables t;
     t.bins = h->d_bins_check;
     t.segs = h->d_segs;
     t.tensors = h->d_tinfo;
-    t.grads = h->d_ptrs;
+    t.grads = h->d_ptrs + (size_t)k * h->n;
     t.nbins = (int32_t)h->L.bins_check.size();
     t.nsegs = (int32_t)h->L.segs.size();
     t.ntensors = h->n;
@@ -617,7 +648,9 @@ static int fail_cuda(mpt_handle* h)
 {
     cudaGetLastError();
     h->broken = true;
-    h->ptrs_uploaded = false;
+    for (auto& sl : h->slot)
+        sl.valid = false;
+    h->cur_slot = -1;
     return MPT_ERR_CUDA;
 }
 
@@ -723,21 +756,25 @@ int mpt_create(const int64_t* sizes, int32_t n, const mpt_config* cfg, void* d_w
               cudaMemset(h->d_ctrl, 0, sizeof(Ctrl)) == cudaSuccess &&
               cudaMemset(h->d_group_tickets, 0, L.off_ptrs - L.off_group_tickets) == cudaSuccess &&
               cudaMemset(h->d_stats, 0, sizeof(StatsBlock)) == cudaSuccess &&
-              cudaMemset(h->d_ptrs, 0, sizeof(void*) * n) == cudaSuccess &&
+              cudaMemset(h->d_ptrs, 0, sizeof(void*) * n * kPtrSlots) == cudaSuccess &&
               cudaMemset(ws + L.off_master, 0, L.total - L.off_master) == cudaSuccess &&
-              cudaHostAlloc(reinterpret_cast<void**>(&h->pinned_ptrs), sizeof(void*) * n, cudaHostAllocDefault) == cudaSuccess &&
               cudaHostAlloc(reinterpret_cast<void**>(&h->mailbox), sizeof(Ctrl), cudaHostAllocDefault) == cudaSuccess &&
               cudaHostAlloc(reinterpret_cast<void**>(&h->hist_box), sizeof(h->hist), cudaHostAllocDefault) == cudaSuccess &&
-              cudaEventCreateWithFlags(&h->ptrs_copied, cudaEventDisableTiming) == cudaSuccess &&
               upload_scaler_state(h, 1.0f, 0) &&
               size_update_grid(h) &&
               cudaDeviceSynchronize() == cudaSuccess;
+    for (auto& sl : h->slot) {
+        if (!ok)
+            break;
+        sl.ptrs.assign(n, nullptr);
+        ok = cudaHostAlloc(reinterpret_cast<void**>(&sl.pinned), sizeof(void*) * n, cudaHostAllocDefault) == cudaSuccess &&
+             cudaEventCreateWithFlags(&sl.copied, cudaEventDisableTiming) == cudaSuccess;
+    }
     if (!ok) {
         cudaGetLastError();
         release(h);
         return MPT_ERR_CUDA;
     }
-    h->last_ptrs.assign(n, nullptr);
     h->stats.scale = h->scale;
     *out = h;
     return MPT_OK;
@@ -844,7 +881,7 @@ int mpt_step_finish(mpt_handle* h, const void* d_partials, int32_t world, float 
         return MPT_ERR_BROKEN;
     if (!finite(lr) || !finite(momentum) || !finite(weight_decay) || !finite(clip))
         return MPT_ERR_INVALID_ARG;
-    if (!h->ptrs_uploaded)
+    if (h->cur_slot < 0)
         return MPT_ERR_INVALID_ARG;  // no check pass queued before
     const int rc = enqueue_step(h, nullptr, true, 0.0f, lr, momentum, weight_decay, clip,
                                 static_cast<cudaStream_t>(cuda_stream), Phase::kShardFinish,

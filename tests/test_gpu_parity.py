@@ -382,6 +382,35 @@ def test_async_steps_follow_the_oracle():
     p.compare_state("after queued steps", exact=True)
 
 
+def test_queued_steps_over_more_buffer_sets_than_cached_tables():
+    """Queued steps that cycle through five gradient buffers, one more than
+    the four pointer tables the handle keeps on the device: steps that reuse
+    a cached table queue no copy, a fifth buffer set rewrites the least
+    recently used table.  Every step must follow the oracle (the device state
+    is compared bit for bit at the end), one of them an overflow."""
+    plan = {7: [(2, 3, 0x7C00)]}
+    cfg = custom([30_000, 1031, 7, 20_000], law=("log2_uniform", -26.0, -4.0), scale0=2.0 ** 12,
+                 growth_interval=3, clip=0.3, steps=14, injections=lambda s: plan.get(s, []))
+    p = Pair(cfg)
+    bufs = [torch.zeros(p.layout.total, dtype=torch.int16, device="cuda") for _ in range(5)]
+    S, skipped = cfg.scale0, 0
+    order = [0, 1, 2, 3, 4, 0, 1, 4, 2, 0, 3, 3, 1, 0]
+    for k, b in enumerate(order, start=1):
+        host = p.grads(k, S)
+        torch.cuda.current_stream().synchronize()      # earlier steps are done with bufs[b]
+        bufs[b].copy_(host)
+        p.opt.step_async(p.layout.views(bufs[b]), cfg.lr, cfg.momentum, cfg.weight_decay, cfg.clip)
+        hv = [v.numpy().view(np.uint16) for v in p.layout.views(host)]
+        ro = oracle.step(p.state, hv, S, cfg.lr, cfg.momentum, cfg.weight_decay, clip=cfg.clip,
+                         cfg=p.ocfg)
+        S = ro["new_scale"]
+        skipped += ro["found_inf"]
+    r = p.opt.wait()
+    assert skipped == 1 and r["new_scale"] == S
+    assert p.opt.stats()["steps"] == len(order) and p.opt.stats()["skipped"] == 1
+    p.compare_state("after steps over five buffer sets", exact=True)
+
+
 def test_stale_total_over_queued_steps():
     """With MPT_FLAG_COUNT_STALE, the running total of stale FP16 elements
     (master moved, rounded copy did not) must count every step queued between
