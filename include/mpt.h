@@ -102,7 +102,7 @@ typedef struct {
     int32_t check_chunk_elems;  /* elements per work bin (one CTA) of the check
                                    pass: a multiple of 2048 in [2048, 2^20];
                                    0 = default: 65536, halved down to 2048
-                                   while the list gives fewer than 2048 bins */
+                                   while the list gives fewer than 592 bins */
     int32_t scaler_mode;      /* MPT_SCALER_DYNAMIC (default) or _DIRECT           */
     float direct_margin;      /* direct mode: margin > 0 (default 2: one bit of
                                  headroom, as the pages suggest)                   */

@@ -19,7 +19,6 @@ constexpr int kMaxPackedSegs = 256;        // tensors per packed bin
 constexpr int kFinishGroup = 64;           // check bins per first-level finish group
 static_assert(kFinishGroup <= kThreads, "one thread per bin of a finish group");
 constexpr int kOneLevelBins = 8 * kThreads; // up to this many check bins: one-level finish
-constexpr int kPackedUnroll = kPackedMaxElems / kThreads;  // elements per thread
 
 enum BinKind : int32_t {
     kChunkBin = 0,   // one contiguous range of one tensor (vectorised)

@@ -560,8 +560,9 @@ __device__ __forceinline__ unsigned int count_nonfinite(const uint16_t* g, int n
 }
 
 // Packed bins: the gradient pointer and offset of each tensor are staged in
-// shared memory once, then every thread handles kPackedUnroll elements with
-// all of its loads issued before any is used.
+// shared memory once, then every thread handles several elements at a time
+// (8 in the check pass, 4 in the update) with all of their loads issued
+// before any is used.
 struct PackedStage {
     int32_t begin[kMaxPackedSegs];
     const uint16_t* gptr[kMaxPackedSegs];

@@ -86,7 +86,7 @@ def test_workspace_bytes():
 
 def test_default_check_bins_follow_the_list_size():
     """Default check bins: 64K elements, halved (to 2048 at least) while the
-    list would give fewer than 296 bins.  Only the check table's size depends
+    list would give fewer than 592 bins.  Only the check table's size depends
     on the chunk, so the explicit chunk whose workspace equals the default's
     is the one the default chose; its neighbours differ by hundreds of bins,
     which the 256-byte region rounding cannot hide."""
@@ -100,10 +100,11 @@ def test_default_check_bins_follow_the_list_size():
                                      ctypes.byref(nb)) == 0
         return nb.value
 
-    cases = [([1 << 20], 2048),                    # 512 bins; 4K would give 256
-             ([10_000_000], 32768),                # 306 bins; 64K would give 153
-             ([19_300_000], 32768),                # 64K gives 295 < 296: halved
-             (W.get("resnet50").sizes, 65536)]     # 390 bins of 64K
+    cases = [([1 << 20], 2048),                    # 512 bins; the floor (4K would give 256)
+             ([10_000_000], 16384),                # 611 bins; 32K would give 306
+             ([38_700_000], 32768),                # 64K gives 591 < 592: halved
+             ([38_900_000], 65536),                # 64K gives 594: kept
+             (W.get("resnet50").sizes, 32768)]     # 780 bins of 32K; 64K would give 390
     for sizes, chunk in cases:
         assert ws(sizes) == ws(sizes, check_chunk_elems=chunk), (sizes[:2], chunk)
         for other in (chunk // 2, chunk * 2):

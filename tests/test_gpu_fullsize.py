@@ -35,7 +35,7 @@ THREADS = min(16, os.cpu_count() or 1)
 
 
 class Sampled:
-    def __init__(self, cfg, n_random=200_000, seed=0, mpt_kw=None, ocfg_kw=None):
+    def __init__(self, cfg, n_random=200_000, seed=0, mpt_kw=None, ocfg_kw=None, shifted=()):
         self.cfg = cfg
         sizes = np.array(cfg.sizes, dtype=np.int64)
         starts = np.concatenate([[0], np.cumsum(sizes)[:-1]])
@@ -44,7 +44,7 @@ class Sampled:
         idx = np.unique(np.concatenate([idx, starts, starts + sizes - 1]))
         self.tensor = np.searchsorted(starts, idx, side="right") - 1
         self.elem = idx - starts[self.tensor]
-        self.layout = W.GradLayout(cfg.sizes)
+        self.layout = W.GradLayout(cfg.sizes, shifted=shifted)
         mpt_kw = mpt_kw or {}
         self.opt = MPT(cfg.sizes, Config(backoff=cfg.backoff, growth=cfg.growth,
                                          growth_interval=cfg.growth_interval, **mpt_kw))
@@ -198,3 +198,12 @@ def test_fullsize_gpt_1p3b():
 def test_fullsize_ragged20k():
     rs = run("ragged20k")
     assert sum(r["found_inf"] for r in rs) >= 20      # 20 injected + natural overflow
+
+
+def test_fullsize_ragged20k_shifted_pointers():
+    """The benchmark's misaligned case: every third gradient tensor starts 2
+    bytes past an aligned address (the check pass's per-thread head, the
+    update's shifted gradient words), queued steps over the full list."""
+    cfg = W.get("ragged20k")
+    rs = run("ragged20k", steps=8, queued=True, shifted=set(range(0, len(cfg.sizes), 3)))
+    assert sum(r["found_inf"] == 0 for r in rs) >= 6
