@@ -8,6 +8,7 @@ rebuild is needed.
 """
 import hashlib
 import os
+import re
 import shutil
 import subprocess
 import sys
@@ -46,13 +47,22 @@ def _digest():
     return h.hexdigest()
 
 
+def _code_only(text):
+    """The source without its comments and with whitespace runs collapsed
+    (the device sources hold no string literal with a comment marker)."""
+    text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", " ", text)
+    return " ".join(text.split())
+
+
 def kernel_digest():
-    """SHA-256 of the device code and its flags (to tell whether a stored
-    profile was taken on the kernels as they are now)."""
+    """SHA-256 of the device code (comments and layout aside) and its flags,
+    to tell whether a stored profile was taken on the kernels as they are
+    now."""
     h = hashlib.sha256()
     for name in ("mpt_kernels.cuh", "mpt_internal.h"):
-        with open(os.path.join(CSRC, name), "rb") as f:
-            h.update(f.read())
+        with open(os.path.join(CSRC, name), encoding="utf-8") as f:
+            h.update(_code_only(f.read()).encode())
     h.update(" ".join(NVCC_FLAGS).encode())
     return h.hexdigest()
 

@@ -102,8 +102,9 @@ __device__ __forceinline__ SqParams sq_params(float S)
 }
 
 // Step result and loss-scale state from the step's totals (one thread): the
-// norm, the clip coefficient, 1/S for the update, the state machine, and the
-// update kernel's counters cleared for this step.
+// norm, the clip coefficient, 1/S for the update, the range counts, the state
+// machine, the previous update's stale count added to the running total, and
+// the update kernel's counters cleared for this step.
 __device__ __forceinline__ void finish_step(Ctrl* c, float S, const SqParams& q,
                                             unsigned long long n_nonfinite, double sumsq,
                                             unsigned int max_mag, bool have_max,

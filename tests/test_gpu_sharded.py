@@ -74,7 +74,7 @@ def test_emulated_ranks_match_the_whole_step(world):
             for k in ("found_inf", "clipped", "new_scale", "clean_run", "grad_norm", "clip_coef",
                       "n_nonfinite"):
                 assert r[k] == res[0][k], k                     # identical on every rank
-        # the range counts come from each rank's update pass: per shard
+        # the range counts come from each rank's check pass: per shard
         assert sum(r["n_zero"] for r in res) == ro["n_zero"]
         assert sum(r["n_subnormal"] for r in res) == ro["n_subnormal"]
         if not ro["found_inf"]:
