@@ -27,7 +27,8 @@ events inside); ``kernels_ms`` from a separate loop of at least 10 steps with
 CUDA events around both kernels of every step (on the launching stream); the
 overflow step (a +inf planted in the gradients: the check pass alone moves
 data) timed apart; ``roofline`` for the update kernel (the dominant one)
-against the measured HBM copy bandwidth.  ``e2e`` (headline) times the same
+against the measured HBM copy bandwidth, with the check kernel inside it, both
+as timed in the step and alone (back to back from a CUDA graph).  ``e2e`` (headline) times the same
 step through the public API with the gradients copied from pinned host memory
 every step and each step's result read back; ``cpu_baseline`` times the CPU
 oracle (single thread) on a bounded leading slice of the workload.
@@ -481,6 +482,35 @@ def measure(cfg, args, R, shift=False, e2e=False, clocks=True):
     }
     if e2e:
         out["e2e"] = measure_e2e(cfg, args, R, opt, sets, ptrs, stream)
+
+    # The check pass on its own: mpt_step_partial queues the check kernel
+    # alone (no finish of the step, no update), replayed back to back from a
+    # CUDA graph -- the kernel's duration without the previous update's dirty
+    # L2 lines to write back and without launch gaps.  Run last: partial
+    # steps leave the handle's range counters to a finish that never comes.
+    opt.step_partial(ptrs[0], stream=stream)
+    opt.wait(stream)
+    side = torch.cuda.Stream(dev)
+    side.wait_stream(stream)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=side):
+        for _ in range(gsteps):
+            opt.step_partial(ptrs[0], stream=side)
+    graph.replay()
+    torch.cuda.synchronize(dev)
+    R.barrier()
+    c0, c1 = ev(), ev()
+    c0.record(stream)
+    for _ in range(greps):
+        graph.replay()
+    c1.record(stream)
+    torch.cuda.synchronize(dev)
+    iso_ms = R.max(c0.elapsed_time(c1)) / (greps * gsteps)
+    del graph
+    iso_gbs = BYTES_CHECK * P / (iso_ms * 1e-3) / 1e9
+    out["roofline"]["check_kernel"]["alone"] = {
+        "ms": iso_ms, "achieved": iso_gbs, "frac": iso_gbs / peak,
+        "how": "check kernel alone, back to back from a CUDA graph (mpt_step_partial)"}
     opt.close()
     del sets
     torch.cuda.synchronize(dev)
