@@ -28,7 +28,9 @@ CUDA events around both kernels of every step (on the launching stream); the
 overflow step (a +inf planted in the gradients: the check pass alone moves
 data) timed apart; ``roofline`` for the update kernel (the dominant one)
 against the measured HBM copy bandwidth, with the check kernel inside it, both
-as timed in the step and alone (back to back from a CUDA graph).  ``e2e`` (headline) times the same
+as timed in the step and alone (L2 cold, from a CUDA graph, without event
+overhead; ``kernels_ms.event_pair_floor`` is what two CUDA events with nothing
+between them read).  ``e2e`` (headline) times the same
 step through the public API with the gradients copied from pinned host memory
 every step and each step's result read back; ``cpu_baseline`` times the CPU
 oracle (single thread) on a bounded leading slice of the workload.
@@ -62,7 +64,10 @@ DEFAULT_EXTRA = "flat1m,resnet50,gpt_1p3b,ragged20k,ragged20k_shift2B"
 BYTES_UPDATE = 20        # per parameter: read g16 2 + w 4 + v 4, write w 4 + v 4 + w16 2
 BYTES_CHECK = 2          # per parameter: read g16
 BYTES_SKIP = 2           # per parameter on an overflow step: the check pass only
-MIN_KERNEL_STEPS = 10    # steps with kernel events, after the headline loop
+MIN_KERNEL_STEPS = 10      # steps with kernel events, after the headline loop
+ALONE_LAUNCHES = 10        # the check pass alone: launches per graph,
+ALONE_REPLAYS = 5          # graph replays per timing,
+SWEEP_BYTES = 512 << 20    # and the read sweep that evicts L2 before each launch
 SKIP_STEPS = 20          # overflow steps timed apart
 NOMINAL_HBM_GBS = 8000.0
 L2_BYTES = 126 * 2 ** 20
@@ -483,34 +488,60 @@ def measure(cfg, args, R, shift=False, e2e=False, clocks=True):
     if e2e:
         out["e2e"] = measure_e2e(cfg, args, R, opt, sets, ptrs, stream)
 
-    # The check pass on its own: mpt_step_partial queues the check kernel
-    # alone (no finish of the step, no update), replayed back to back from a
-    # CUDA graph -- the kernel's duration without the previous update's dirty
-    # L2 lines to write back and without launch gaps.  Run last: partial
-    # steps leave the handle's range counters to a finish that never comes.
-    opt.step_partial(ptrs[0], stream=stream)
-    opt.wait(stream)
+    # The check pass on its own, with L2 cold: before each launch a read-only
+    # sweep of a 512 MB buffer (four times L2) evicts the gradients without
+    # leaving dirty lines behind.  A CUDA graph of (sweep, check) pairs minus
+    # a graph of the sweeps alone gives the check's cost per launch (its
+    # launch included, no event overhead), and the median of three such
+    # differences is reported.  mpt_step_partial queues the check kernel
+    # alone (no finish of the step, no update).  Run last: partial steps
+    # leave the handle's range counters to a finish that never comes.
+    sweep = torch.ones(SWEEP_BYTES // 4, dtype=torch.float32, device=dev)
+    sink = torch.empty((), dtype=torch.float32, device=dev)
     side = torch.cuda.Stream(dev)
     side.wait_stream(stream)
-    graph = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(graph, stream=side):
-        for _ in range(gsteps):
-            opt.step_partial(ptrs[0], stream=side)
-    graph.replay()
-    torch.cuda.synchronize(dev)
-    R.barrier()
-    c0, c1 = ev(), ev()
-    c0.record(stream)
-    for _ in range(greps):
+
+    def sweep_graph_ms(with_check):
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=side):
+            for k in range(ALONE_LAUNCHES):
+                torch.sum(sweep, dim=0, out=sink)
+                if with_check:
+                    opt.step_partial(ptrs[k % len(ptrs)], stream=side)
         graph.replay()
-    c1.record(stream)
+        torch.cuda.synchronize(dev)
+        R.barrier()
+        c0, c1 = ev(), ev()
+        c0.record(stream)
+        for _ in range(ALONE_REPLAYS):
+            graph.replay()
+        c1.record(stream)
+        torch.cuda.synchronize(dev)
+        del graph
+        return R.max(c0.elapsed_time(c1)) / (ALONE_REPLAYS * ALONE_LAUNCHES)
+
+    diffs = []
+    for _ in range(3):
+        with_check = sweep_graph_ms(True)
+        diffs.append(with_check - sweep_graph_ms(False))
+    iso_ms = statistics.median(diffs)
+    # what a pair of CUDA events with nothing between them reads after such a
+    # sweep: the part of an event-timed kernel duration that is not the kernel
+    floor = []
+    for _ in range(10):
+        torch.sum(sweep, dim=0, out=sink)
+        f0, f1 = ev(), ev()
+        f0.record(stream)
+        f1.record(stream)
+        floor.append((f0, f1))
     torch.cuda.synchronize(dev)
-    iso_ms = R.max(c0.elapsed_time(c1)) / (greps * gsteps)
-    del graph
+    out["kernels_ms"]["event_pair_floor"] = R.max(statistics.median(a.elapsed_time(b) for a, b in floor))
+    del sweep, sink
     iso_gbs = BYTES_CHECK * P / (iso_ms * 1e-3) / 1e9
     out["roofline"]["check_kernel"]["alone"] = {
         "ms": iso_ms, "achieved": iso_gbs, "frac": iso_gbs / peak,
-        "how": "check kernel alone, back to back from a CUDA graph (mpt_step_partial)"}
+        "how": ("check kernel alone with L2 cold: CUDA graph of %d (512 MB read sweep, "
+                "mpt_step_partial) pairs minus the sweeps alone, median of 3" % ALONE_LAUNCHES)}
     opt.close()
     del sets
     torch.cuda.synchronize(dev)

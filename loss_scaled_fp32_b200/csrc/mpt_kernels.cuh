@@ -513,24 +513,25 @@ __device__ __forceinline__ CtaTotals block_totals(double x, unsigned int nz, uns
 }
 
 // This thread's share of the per-bin partials, k = threadIdx.x + i*kThreads in
-// increasing i, with eight loads issued before they are added (the same order
-// of additions as one load at a time).
+// increasing i, eight loads issued before they are added (the same order of
+// additions as one load at a time).  Slots past n read as +0.0, which leaves
+// the running sum unchanged: the partials are non-negative, +inf or NaN, so
+// the sum is never -0.0.  The last batch is thereby one round of loads too.
 __device__ __forceinline__ double sum_partials(const double* partials, int n)
 {
     constexpr int kU = 8;
     double x = 0.0;
-    int k = threadIdx.x;
-    for (; k + (kU - 1) * kThreads < n; k += kU * kThreads) {
+    for (int k = threadIdx.x; k < n; k += kU * kThreads) {
         double p[kU];
 #pragma unroll
-        for (int i = 0; i < kU; ++i)
-            p[i] = __ldcg(partials + k + i * kThreads);
+        for (int i = 0; i < kU; ++i) {
+            const int j = k + i * kThreads;
+            p[i] = j < n ? __ldcg(partials + j) : 0.0;
+        }
 #pragma unroll
         for (int i = 0; i < kU; ++i)
             x += p[i];
     }
-    for (; k < n; k += kThreads)
-        x += __ldcg(partials + k);
     return x;
 }
 
