@@ -29,8 +29,9 @@ overflow step (a +inf planted in the gradients: the check pass alone moves
 data) timed apart; ``roofline`` for the update kernel (the dominant one)
 against the measured HBM copy bandwidth, with the check kernel inside it, both
 as timed in the step and alone (L2 cold, from a CUDA graph, without event
-overhead; ``kernels_ms.event_pair_floor`` is what two CUDA events with nothing
-between them read).  ``e2e`` (headline) times the same
+overhead, in the sharded step's form that also adds its own partials;
+``kernels_ms.event_pair_floor`` is what two CUDA events with nothing between
+them read).  ``e2e`` (headline) times the same
 step through the public API with the gradients copied from pinned host memory
 every step and each step's result read back; ``cpu_baseline`` times the CPU
 oracle (single thread) on a bounded leading slice of the workload.
@@ -494,8 +495,11 @@ def measure(cfg, args, R, shift=False, e2e=False, clocks=True):
     # a graph of the sweeps alone gives the check's cost per launch (its
     # launch included, no event overhead), and the median of three such
     # differences is reported.  mpt_step_partial queues the check kernel
-    # alone (no finish of the step, no update).  Run last: partial steps
-    # leave the handle's range counters to a finish that never comes.
+    # alone as the sharded step runs it: it also adds its own partials
+    # (atomic tickets, the 32-byte record), which a whole step leaves to the
+    # update kernel, so it is an upper bound of the check in a whole step.
+    # Run last: partial steps leave the handle's range counters to a finish
+    # that never comes.
     sweep = torch.ones(SWEEP_BYTES // 4, dtype=torch.float32, device=dev)
     sink = torch.empty((), dtype=torch.float32, device=dev)
     side = torch.cuda.Stream(dev)
@@ -541,7 +545,8 @@ def measure(cfg, args, R, shift=False, e2e=False, clocks=True):
     out["roofline"]["check_kernel"]["alone"] = {
         "ms": iso_ms, "achieved": iso_gbs, "frac": iso_gbs / peak,
         "how": ("check kernel alone with L2 cold: CUDA graph of %d (512 MB read sweep, "
-                "mpt_step_partial) pairs minus the sweeps alone, median of 3" % ALONE_LAUNCHES)}
+                "mpt_step_partial) pairs minus the sweeps alone, median of 3; the sharded "
+                "step's form of the pass, which also adds its own partials" % ALONE_LAUNCHES)}
     opt.close()
     del sets
     torch.cuda.synchronize(dev)

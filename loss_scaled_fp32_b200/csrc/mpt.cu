@@ -2,16 +2,18 @@
 //
 // One step = two kernel launches on the caller's stream and, for the
 // waiting call, one 384-byte read-back of the control block:
-//   check_kernel  (2 B/param)  overflow flag, sum of squares, range counts,
-//                              two-level finish -> norm, clip coefficient,
-//                              next S
-//   update_kernel (20 B/param) fused unscale/clip/decay/momentum/master/FP16
+//   check_kernel  (2 B/param)  overflow flag, sum of squares, range counts as
+//                              per-bin (or per-group) partials
+//   update_kernel (20 B/param) every CTA adds the partials (norm, clip
+//                              coefficient, overflow flag), CTA 0 writes the
+//                              result and the next S; then the fused
+//                              unscale/clip/decay/momentum/master/FP16 update
 //                              over a persistent grid; on an overflow step
-//                              each CTA reads the flag and exits
+//                              each CTA exits after the sum
 // The launch order alone carries the check result to the update, so no host
-// decision sits between the two kernels.  The loss-scale state machine runs in
-// the check kernel's last CTA and keeps S on the device, so that steps can be
-// queued without waiting (mpt_step_async); the host mirrors it on read-back.
+// decision sits between the two kernels.  The loss-scale state machine runs on
+// the device and keeps S there, so that steps can be queued without waiting
+// (mpt_step_async); the host mirrors it on read-back.
 #include <cuda_runtime.h>
 #include <nvtx3/nvToolsExt.h>
 
@@ -545,6 +547,7 @@ static int enqueue_step(mpt_handle* h, const void* const* d_grads_half, bool sca
     ca.scaler.direct_margin = h->cfg.direct_margin;
     ca.stats = h->d_stats;
     ca.partial_out = phase == Phase::kShardCheck ? h->d_partial_rec : nullptr;
+    ca.defer_finish = phase == Phase::kWhole ? 1 : 0;
 
     UpdateArgs ua;
     ua.t = t;
@@ -558,6 +561,16 @@ static int enqueue_step(mpt_handle* h, const void* const* d_grads_half, bool sca
     ua.mu = momentum;
     ua.wd = weight_decay;
     ua.eps = h->cfg.eps;
+    {
+        const int nbc = (int)h->L.bins_check.size();
+        const bool one_level = nbc <= kOneLevelBins;
+        ua.fin_src = phase == Phase::kWhole ? (one_level ? h->d_partials : h->d_groups) : nullptr;
+        ua.fin_n = one_level ? nbc : (nbc + kFinishGroup - 1) / kFinishGroup;
+    }
+    ua.stats_level = stats_level(h);
+    ua.clip = clip;
+    ua.scaler = ca.scaler;
+    ua.stats = h->d_stats;
 
     const bool checked = (h->cfg.flags & MPT_FLAG_CHECKED) != 0;
     const bool stale = (h->cfg.flags & MPT_FLAG_COUNT_STALE) != 0;

@@ -3,11 +3,17 @@
 //   check_kernel   one pass over the FP16 gradients: overflow check (Step 6 of
 //                  "The Integrated Training Procedure (Figure 1)"), sum of
 //                  squares of the unscaled gradients (global-L2 clip), zero
-//                  and subnormal counts, with a deterministic two-level
-//                  finish that writes the step result
-//   update_kernel  the fused per-element update (Steps 5 and 7, weight decay,
-//                  clip, FP16 copy) over a persistent grid; on an overflow
-//                  step every CTA reads the flag and exits
+//                  and subnormal counts, as per-bin (beyond 2 048 bins
+//                  per-group) partial sums
+//   update_kernel  adds those partials in a fixed order (every CTA the same
+//                  sum; CTA 0 writes the step result and advances the loss
+//                  scale), then the fused per-element update (Steps 5 and 7,
+//                  weight decay, clip, FP16 copy) over a persistent grid; on
+//                  an overflow step every CTA exits after the sum
+//
+// The sharded step's check pass (mpt_step_partial) instead finishes its own
+// partials by atomic tickets into a 32-byte record, and finish_kernel
+// combines the ranks' records before the update.
 //   refresh_kernel FP16 copy = round-to-nearest-even(master) (Step 1)
 //
 // All three are HBM-bound streaming kernels on the CUDA cores: there is no
@@ -65,6 +71,8 @@ struct CheckArgs {
     StatsBlock* stats;    // statistics mode only
     Partial* partial_out; // sharded step: write this shard's totals here and
                           // leave the finish to finish_kernel; nullptr: finish
+    int32_t defer_finish; // 1: leave the partials to the update kernel, which
+                          // adds them and finishes the step (whole steps)
 };
 
 struct UpdateArgs {
@@ -77,6 +85,15 @@ struct UpdateArgs {
     float mu;
     float wd;
     float eps;            // Adagrad only
+    // whole steps: the check kernel's partial sums (per bin, or per group of
+    // kFinishGroup bins beyond kOneLevelBins bins), added by every CTA; the
+    // step is finished by CTA 0.  nullptr: the result is already in ctrl.
+    const double* fin_src;
+    int32_t fin_n;
+    int32_t stats_level;  // kNoStats, kMaxOnly or kMaxHist
+    float clip;
+    ScalerParams scaler;
+    StatsBlock* stats;
 };
 
 // What the squares need from S: the binary32 reciprocal 1/S and, when S is a
@@ -108,7 +125,8 @@ __device__ __forceinline__ SqParams sq_params(float S)
 __device__ __forceinline__ void finish_step(Ctrl* c, float S, const SqParams& q,
                                             unsigned long long n_nonfinite, double sumsq,
                                             unsigned int max_mag, bool have_max,
-                                            unsigned int err, float clip, const ScalerParams& sp)
+                                            unsigned int err, float clip, const ScalerParams& sp,
+                                            bool deferred = false)
 {
     const bool found = n_nonfinite != 0;
     const double norm = found ? __longlong_as_double(0x7ff0000000000000ll) : sqrt(sumsq);
@@ -125,9 +143,17 @@ __device__ __forceinline__ void finish_step(Ctrl* c, float S, const SqParams& q,
     c->found_inf = found ? 1 : 0;
     c->clipped = clipped ? 1 : 0;
     c->coef = clipped ? __double2float_rn((double)clip / norm) : 1.0f;
-    c->inv_scale = q.inv_scale;
-    c->scale_used = S;
-    c->error = err;
+    if (deferred) {
+        // S, 1/S, the cleared error word, the update's bin counter and the
+        // stale total were set by the check kernel's CTA 0; the update's own
+        // CTAs may be adding error bits right now
+        if (err)
+            atomicOr(&c->error, err);
+    } else {
+        c->inv_scale = q.inv_scale;
+        c->scale_used = S;
+        c->error = err;
+    }
     // Loss-scale state machine: on overflow skip and multiply S by beta;
     // dynamic mode: after growth_interval consecutive clean steps multiply S
     // by alpha; direct mode: S = 65504 / (margin * max|g|) of this step
@@ -162,8 +188,10 @@ __device__ __forceinline__ void finish_step(Ctrl* c, float S, const SqParams& q,
     // count joins the running total; the update's accumulators start over
     c->n_zero = atomicExch(&c->zero_acc, 0ull);
     c->n_subnormal = atomicExch(&c->subnormal_acc, 0ull);
-    c->stale_total += atomicExch(&c->stale_acc, 0ull);
-    c->upd_next = 0;
+    if (!deferred) {
+        c->stale_total += atomicExch(&c->stale_acc, 0ull);
+        c->upd_next = 0;
+    }
 }
 
 
@@ -633,8 +661,9 @@ __global__ void __launch_bounds__(kThreads, kStats == kMaxHist ? 4 : 8) check_ke
     const Tables& t = a.t;
     const Bin bin = t.bins[blockIdx.x];
     // S of these gradients: the host's, or the device state the previous
-    // step left (it changes only in this kernel's last CTA, after every other
-    // CTA has finished reading it)
+    // step left (written only by the kernel that finishes a step: the update
+    // kernel before this one, or this kernel's last CTA in a sharded step,
+    // after every other CTA has finished reading it)
     float S;
     SqParams q;
     if (a.scale_on_device) {
@@ -648,6 +677,19 @@ __global__ void __launch_bounds__(kThreads, kStats == kMaxHist ? 4 : 8) check_ke
         q.inv_scale = a.host_inv;
         q.sq_unscale = a.host_sq_unscale;
         q.pow2 = a.host_pow2 != 0;
+    }
+    if (a.defer_finish && blockIdx.x == 0 && threadIdx.x == 0) {
+        // For the update kernel, which finishes this step: S and 1/S of
+        // these gradients, a cleared error word, its bin counter at zero, and
+        // the last update's stale count moved into the total (that update
+        // has completed; nothing else touches these fields during the pass).
+        Ctrl* c = a.ctrl;
+        c->inv_scale = q.inv_scale;
+        c->scale_used = S;
+        c->error = 0u;
+        c->upd_next = 0u;
+        c->stale_total += c->stale_acc;
+        c->stale_acc = 0ull;
     }
     SqAcc s;
     RangeCounts rc;
@@ -745,7 +787,11 @@ __global__ void __launch_bounds__(kThreads, kStats == kMaxHist ? 4 : 8) check_ke
             atomicMax(&a.ctrl->max_mag_acc, mx);
     }
     if (threadIdx.x == 0) {
-        a.partials[blockIdx.x] = part;
+        // deferred finish: a bin that holds an inf/NaN gradient leaves NaN,
+        // so the total is NaN exactly when the step overflowed (every other
+        // partial is in [0, +inf]: +inf only from a binary32 product that a
+        // huge 1/S overflowed, and a sum of those is never NaN)
+        a.partials[blockIdx.x] = (a.defer_finish && nf) ? __longlong_as_double(0x7ff8000000000000ll) : part;
         if (nf)
             atomicAdd(&a.ctrl->nonfinite_acc, (unsigned long long)nf);
         if (valid) {
@@ -769,6 +815,8 @@ __global__ void __launch_bounds__(kThreads, kStats == kMaxHist ? 4 : 8) check_ke
     // Either way the additions follow a fixed pattern (bin order within a
     // thread's share, a fixed tree across threads), whichever CTA is last.
     __syncthreads();  // every write of this CTA precedes its ticket
+    if (a.defer_finish && (int)gridDim.x <= kOneLevelBins)
+        return;  // the update kernel adds the per-bin partials
     double sumsq;
     if ((int)gridDim.x <= kOneLevelBins) {
         if (threadIdx.x == 0) {
@@ -795,6 +843,14 @@ __global__ void __launch_bounds__(kThreads, kStats == kMaxHist ? 4 : 8) check_ke
         const double gsum = block_sum(
             threadIdx.x < g_len ? __ldcg(a.partials + g_begin + threadIdx.x) : 0.0, s_red);
         const int ngroups = ((int)gridDim.x + kFinishGroup - 1) / kFinishGroup;
+        if (a.defer_finish) {
+            // the update kernel adds the group sums
+            if (threadIdx.x == 0) {
+                a.group_partials[grp] = gsum;
+                a.group_tickets[grp] = 0;
+            }
+            return;
+        }
         if (threadIdx.x == 0) {
             a.group_partials[grp] = gsum;
             a.group_tickets[grp] = 0;
@@ -1068,15 +1124,18 @@ __device__ __forceinline__ void update_range(const uint16_t* g, float* w, float*
 // takes bin c first (counted from the end: the check kernel read the last
 // bins last, so their gradients are the ones still in L2) and then, each time
 // it finishes a bin, claims the next one, gridDim.x + k for the k-th claim,
-// from a counter that the check kernel's last CTA resets every step: bins
-// start in order, and an SM that streams faster takes more of them.  An
-// overflow step costs one flag read per CTA.
+// from a counter that the check kernel resets every step: bins start in
+// order, and an SM that streams faster takes more of them.  An overflow step
+// costs each CTA one sum of the check kernel's partials.
 template <int kOpt, bool kStale, bool kChecked>
 __global__ void __launch_bounds__(kThreads, kOpt == kOptAdagrad ? 3 : 4) update_kernel(UpdateArgs a)
 {
     __shared__ PackedStage st;
     __shared__ int s_next[2];
     __shared__ unsigned int s_ured[kWarps];
+    __shared__ double s_red[kWarps];
+    __shared__ int s_found;
+    __shared__ float s_coef;
 
     const Tables& t = a.t;
     const int nb = t.nbins;
@@ -1110,15 +1169,52 @@ __global__ void __launch_bounds__(kThreads, kOpt == kOptAdagrad ? 3 : 4) update_
     // Wait until the check kernel has finished and its result is visible
     // (returns at once when this grid was launched without overlap).
     asm volatile("griddepcontrol.wait;" ::: "memory");
-    // the check result, read past L1 (the hint above may have cached the
-    // line before the check kernel's last CTA wrote it)
     Ctrl* c = a.ctrl;
-    if (__ldcg(&c->found_inf) != 0) {
-        // Overflow step (Step 6): master, momentum and FP16 copy stay as they
-        // are.  The flag is the same for every thread of the grid.
-        return;
+    float coef;
+    if (a.fin_src) {
+        // Whole step: add the check kernel's partials (the same order of
+        // additions in every CTA, so every CTA obtains the same sum); NaN
+        // means some gradient was inf/NaN.  CTA 0 also finishes the step:
+        // the result, the loss-scale state, the accumulators cleared (this
+        // CTA is their only reader).
+        const double sumsq = block_sum(sum_partials(a.fin_src, a.fin_n), s_red);
+        if (threadIdx.x == 0) {
+            const bool found = isnan(sumsq);
+            const double norm = found ? __longlong_as_double(0x7ff0000000000000ll) : sqrt(sumsq);
+            const bool clipped = !found && a.clip > 0.0f && norm > (double)a.clip;
+            s_found = found ? 1 : 0;
+            s_coef = clipped ? __double2float_rn((double)a.clip / norm) : 1.0f;
+            if (blockIdx.x == 0) {
+                if (a.stats_level == kMaxHist)
+                    for (int k = 0; k < 32; ++k)
+                        a.stats->hist[k] = atomicExch(&a.stats->hist_acc[k], 0ull);
+                const unsigned long long n_nonfinite = atomicExch(&c->nonfinite_acc, 0ull);
+                const unsigned int err = atomicExch(&c->error_acc, 0u);
+                const bool have_max = a.stats_level != kNoStats;
+                const unsigned int mm = have_max ? atomicExch(&c->max_mag_acc, 0u) : 0u;
+                SqParams q;
+                q.inv_scale = __ldcg(&c->inv_scale);
+                q.sq_unscale = 0.0;
+                q.pow2 = false;
+                finish_step(c, __ldcg(&c->scale_used), q, n_nonfinite, sumsq, mm, have_max, err,
+                            a.clip, a.scaler, true);
+            }
+        }
+        __syncthreads();
+        if (s_found)
+            return;  // Step 6: master, momentum and FP16 copy stay as they are
+        coef = s_coef;
+    } else {
+        // the result finish_kernel left, read past L1 (the hint above may
+        // have cached the line before it was written)
+        if (__ldcg(&c->found_inf) != 0) {
+            // Overflow step (Step 6): master, momentum and FP16 copy stay as
+            // they are.  The flag is the same for every thread of the grid.
+            return;
+        }
+        coef = __ldcg(&c->coef);
     }
-    const UpdParams p{__ldcg(&c->inv_scale), __ldcg(&c->coef), a.lr, a.mu, a.wd, a.eps};
+    const UpdParams p{__ldcg(&c->inv_scale), coef, a.lr, a.mu, a.wd, a.eps};
     uint32_t stale = 0;
     bool bad = false;
 

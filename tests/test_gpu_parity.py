@@ -162,6 +162,29 @@ def test_huge_inverse_scale_overflows_products_not_the_check():
     p.compare_state("huge 1/S", exact=True)
 
 
+def test_huge_inverse_scale_with_one_inf_gradient_is_skipped():
+    """The same S = 2^-120, now with one +inf gradient in the second tensor:
+    some bins' sums are +inf from overflowing products alone, one bin holds a
+    non-finite gradient.  Only the latter makes the step an overflow step: it
+    is skipped, the non-finite count is exact and the state stays bitwise
+    unchanged, as in the oracle."""
+    cfg = custom([70_000, 3001], law=("log2_uniform", 112.0, 130.0), scale0=2.0 ** -120, steps=1)
+    p = Pair(cfg)
+    host = p.grads(1, p.scale)
+    host[p.layout.offsets[1] + 1234] = 0x7C00
+    p.flat.copy_(host)
+    hv = [v.numpy().view(np.uint16) for v in p.layout.views(host)]
+    r = p.opt.step(p.gviews, p.scale, cfg.lr, cfg.momentum, cfg.weight_decay, 1.0)
+    ro = oracle.step(p.state, hv, p.scale, cfg.lr, cfg.momentum, cfg.weight_decay, clip=1.0,
+                     cfg=p.ocfg)
+    assert ro["found_inf"] == 1 and r["found_inf"] == 1
+    assert r["n_nonfinite"] == ro["n_nonfinite"] == 1
+    assert math.isinf(r["grad_norm"]) and r["clip_coef"] == 1.0
+    assert r["n_zero"] == ro["n_zero"] and r["n_subnormal"] == ro["n_subnormal"]
+    assert r["new_scale"] == ro["new_scale"]
+    p.compare_state("huge 1/S, one inf", exact=True)
+
+
 def test_steps_write_nothing_outside_the_tensors():
     """Guard canaries: every byte of the master, momentum and FP16 arenas that
     belongs to no tensor (the 16-element padding after each tensor and the
