@@ -10,11 +10,11 @@
 //                  scale), then the fused per-element update (Steps 5 and 7,
 //                  weight decay, clip, FP16 copy) over a persistent grid; on
 //                  an overflow step every CTA exits after the sum
+//   refresh_kernel FP16 copy = round-to-nearest-even(master) (Step 1)
 //
 // The sharded step's check pass (mpt_step_partial) instead finishes its own
 // partials by atomic tickets into a 32-byte record, and finish_kernel
 // combines the ranks' records before the update.
-//   refresh_kernel FP16 copy = round-to-nearest-even(master) (Step 1)
 //
 // All three are HBM-bound streaming kernels on the CUDA cores: there is no
 // contraction, so no tensor-core path.  Per parameter the check reads 2 B and
@@ -184,8 +184,9 @@ __device__ __forceinline__ void finish_step(Ctrl* c, float S, const SqParams& q,
     c->next_pow2 = nq.pow2 ? 1 : 0;
     c->clean_run = clean;
     c->steps_total += 1;
-    // range counts of this step's check pass; the previous update's stale
-    // count joins the running total; the update's accumulators start over
+    // range counts of this step's check pass; in a sharded step also the
+    // previous update's stale count joins the running total and the update's
+    // bin counter starts over (a whole step's check kernel did both already)
     c->n_zero = atomicExch(&c->zero_acc, 0ull);
     c->n_subnormal = atomicExch(&c->subnormal_acc, 0ull);
     if (!deferred) {
