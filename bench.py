@@ -422,8 +422,8 @@ def measure(cfg, args, R, shift=False, e2e=False, clocks=True):
 
     # overflow (skipped) steps, reported apart: one +inf planted in the
     # gradients, so every step takes the skip path -- the check pass reads
-    # the gradients, the update grid reads the flag and exits -- and halves S
-    # on the device
+    # the gradients, each update CTA adds the check's partials, finds NaN and
+    # exits -- and halves S on the device
     flat0 = sets[0]
     at = layout.offsets[0]
     saved = flat0[at].item()
