@@ -18,7 +18,8 @@ import pytest
 import torch
 
 import oracle
-from loss_scaled_fp32_b200 import MPT, MPT_PARTIAL_BYTES, Config, shard_len
+from loss_scaled_fp32_b200 import (MPT, MPT_FLAG_GRAD_STATS, MPT_PARTIAL_BYTES, MPT_SCALER_DIRECT,
+                                   Config, shard_len)
 
 pytestmark = pytest.mark.gpu
 
@@ -95,6 +96,50 @@ def test_emulated_ranks_match_the_whole_step(world):
                 assert hw.tobytes() == state.w16[0][sl].tobytes()
     for h in shards:
         h.close()
+
+
+@pytest.mark.parametrize("n,chunk,flags,mode", [
+    (3_000_017, 0, 0, 0),                                       # 733 check bins: one level
+    (5_000_011, 2048, MPT_FLAG_GRAD_STATS, MPT_SCALER_DIRECT),  # 2 442 bins: two levels
+])
+def test_whole_step_and_one_rank_sharded_step_agree_bit_for_bit(n, chunk, flags, mode):
+    """A whole step is finished by the update kernel (every CTA adds the check
+    kernel's partials, CTA 0 writes the result and the next S); a one-rank
+    sharded step by the check kernel's ticket finish, its 32-byte record and
+    finish_kernel.  Both add the same partials in the same order, so from the
+    same state and gradients they must leave the same bits -- results, loss
+    scale, histogram, master, momentum and FP16 copy -- over clean, clipped
+    and overflowing steps."""
+    rng = np.random.default_rng(n)
+    master = rng.normal(0, 0.05, n).astype(np.float32)
+    cfg = Config(growth_interval=2, check_chunk_elems=chunk, flags=flags, scaler_mode=mode)
+    a, b = MPT([n], cfg), MPT([n], cfg)
+    for h in (a, b):
+        h.master(0).copy_(torch.from_numpy(master))
+        h.refresh_half()
+        h.set_scaler_state(2.0 ** 12, 0)
+    g = torch.empty(n, dtype=torch.int16, device="cuda")
+    seen = set()
+    for step in range(6):
+        host = _grads(rng, n, n)
+        if step == 3:
+            host[n // 2] = 0x7C00
+        g.copy_(torch.from_numpy(host.view(np.int16)))
+        a.step_async([g], 0.01, 0.9, 1e-4, clip=0.5)
+        ra = a.wait()
+        rec = b.step_partial([g]).clone()
+        b.step_finish(rec, 1, 0.01, 0.9, 1e-4, clip=0.5)
+        rb = b.wait()
+        assert ra == rb, step
+        seen.add("overflow" if ra["found_inf"] else "clipped" if ra["clipped"] else "clean")
+        assert torch.equal(a.master(0).view(torch.int32), b.master(0).view(torch.int32)), step
+        assert torch.equal(a.momentum(0).view(torch.int32), b.momentum(0).view(torch.int32)), step
+        assert torch.equal(a.w16(0), b.w16(0)), step
+        if flags & MPT_FLAG_GRAD_STATS:
+            assert a.grad_histogram() == b.grad_histogram(), step
+    assert {"overflow", "clipped"} <= seen
+    a.close()
+    b.close()
 
 
 def test_sharded_optimizer_single_rank_nccl():
