@@ -261,9 +261,9 @@ int mpt_device_scale(const mpt_handle* h, float** d_scale);
  *      of squares, non-finite count, largest finite |g16|, error bits);
  *   3. the caller all-gathers the records of all ranks, in rank order, into
  *      one device array (16-byte aligned);
- *   4. mpt_step_finish adds the records in rank order (so every rank gets
- *      bit-identical totals and the same next S), finishes the step and
- *      queues the update of the shard;
+ *   4. mpt_step_finish queues the update of the shard, which first adds the
+ *      records in rank order (so every rank gets bit-identical totals and the
+ *      same next S) and finishes the step;
  *   5. the caller all-gathers the FP16 copies of the shards.
  * Only 32 bytes per rank cross between the two kernels of a step.  The
  * halves are not timed by mpt_set_timing; mpt_wait returns the last result:
@@ -285,8 +285,9 @@ int mpt_step_partial(mpt_handle* h, const void* const* d_grads_half, void* cuda_
                      void** d_partial);
 
 /* Phase 4: d_partials = device array of `world` records in rank order;
- * finishes the step (norm, clip coefficient, loss-scale state) and queues the
- * update over the gradients of the preceding mpt_step_partial.
+ * queues the update over the gradients of the preceding mpt_step_partial,
+ * which first adds the records and finishes the step (norm, clip
+ * coefficient, loss-scale state).
  * Errors: MPT_ERR_INVALID_ARG (no check pass queued, misaligned records),
  * MPT_ERR_CUDA, MPT_ERR_BROKEN. */
 int mpt_step_finish(mpt_handle* h, const void* d_partials, int32_t world, float lr,

@@ -447,8 +447,8 @@ static void launch_update_any(const mpt_handle* h, const UpdateArgs& ua, bool st
 }
 
 // What enqueue_step queues: the whole step, or one half of a sharded step
-// (the check pass writing this shard's record / the combine-and-finish kernel
-// followed by the update).
+// (the check pass writing this shard's record / the update, which adds the
+// ranks' records and finishes the step).
 enum class Phase { kWhole, kShardCheck, kShardFinish };
 
 // An NVTX range around the host work of one call (named ranges for a
@@ -537,17 +537,8 @@ static int enqueue_step(mpt_handle* h, const void* const* d_grads_half, bool sca
         ca.host_pow2 = hp.pow2;
     }
     ca.scale_on_device = scale_on_device ? 1 : 0;
-    ca.clip = clip;
-    ca.scaler.backoff = h->cfg.backoff;
-    ca.scaler.growth = h->cfg.growth;
-    ca.scaler.growth_interval = h->cfg.growth_interval;
-    ca.scaler.min_scale = h->cfg.min_scale;
-    ca.scaler.max_scale = h->cfg.max_scale;
-    ca.scaler.mode = h->cfg.scaler_mode;
-    ca.scaler.direct_margin = h->cfg.direct_margin;
     ca.stats = h->d_stats;
     ca.partial_out = phase == Phase::kShardCheck ? h->d_partial_rec : nullptr;
-    ca.defer_finish = phase == Phase::kWhole ? 1 : 0;
 
     UpdateArgs ua;
     ua.t = t;
@@ -562,32 +553,34 @@ static int enqueue_step(mpt_handle* h, const void* const* d_grads_half, bool sca
     ua.wd = weight_decay;
     ua.eps = h->cfg.eps;
     {
+        // whole step: the check kernel's per-bin (or per-group) partials;
+        // sharded step: the ranks' records
         const int nbc = (int)h->L.bins_check.size();
         const bool one_level = nbc <= kOneLevelBins;
-        ua.fin_src = phase == Phase::kWhole ? (one_level ? h->d_partials : h->d_groups) : nullptr;
-        ua.fin_n = one_level ? nbc : (nbc + kFinishGroup - 1) / kFinishGroup;
+        const bool whole = phase == Phase::kWhole;
+        ua.fin_partials = whole ? (one_level ? h->d_partials : h->d_groups) : nullptr;
+        ua.fin_n = whole ? (one_level ? nbc : (nbc + kFinishGroup - 1) / kFinishGroup) : 0;
+        ua.fin_records = whole ? nullptr : static_cast<const Partial*>(d_parts);
+        ua.fin_world = whole ? 0 : world;
     }
     ua.stats_level = stats_level(h);
     ua.clip = clip;
-    ua.scaler = ca.scaler;
+    ua.scaler.backoff = h->cfg.backoff;
+    ua.scaler.growth = h->cfg.growth;
+    ua.scaler.growth_interval = h->cfg.growth_interval;
+    ua.scaler.min_scale = h->cfg.min_scale;
+    ua.scaler.max_scale = h->cfg.max_scale;
+    ua.scaler.mode = h->cfg.scaler_mode;
+    ua.scaler.direct_margin = h->cfg.direct_margin;
     ua.stats = h->d_stats;
 
     const bool checked = (h->cfg.flags & MPT_FLAG_CHECKED) != 0;
     const bool stale = (h->cfg.flags & MPT_FLAG_COUNT_STALE) != 0;
     if (phase != Phase::kWhole) {  // sharded step halves (not timed)
-        if (phase == Phase::kShardCheck) {
+        if (phase == Phase::kShardCheck)
             launch_check_level(h, ca, checked, st);
-        } else {
-            FinishArgs fa;
-            fa.parts = static_cast<const Partial*>(d_parts);
-            fa.world = world;
-            fa.have_max = stats_on(h) ? 1 : 0;
-            fa.ctrl = h->d_ctrl;
-            fa.clip = clip;
-            fa.scaler = ca.scaler;
-            finish_kernel<<<1, 32, 0, st>>>(fa);
+        else
             launch_update_any(h, ua, stale, checked, st);
-        }
         return cudaGetLastError() == cudaSuccess ? MPT_OK : MPT_ERR_CUDA;
     }
 

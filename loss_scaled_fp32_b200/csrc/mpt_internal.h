@@ -54,9 +54,9 @@ struct __align__(16) TensorInfo {
 };
 
 // Device control block.  The check kernel accumulates into the *_acc fields;
-// the kernel that finishes the step (CTA 0 of the update kernel in a whole
-// step; in a sharded step the check kernel's last CTA and finish_kernel)
-// turns them into the step result and clears them for the next step.  The two
+// CTA 0 of the update kernel turns them (in a sharded step: the ranks'
+// records, which the check kernel's last CTA drew from them) into the step
+// result and clears them for the next step.  The two
 // kernels' atomic accumulators and the fields that every CTA reads when it
 // starts (S, 1/S, the skip flag, the clip coefficient) sit on three separate
 // 128-byte lines, so that a CTA's first read never queues behind the other
@@ -72,15 +72,14 @@ struct __align__(128) Ctrl {
     unsigned long long subnormal_acc;  // FP16 gradients with 0 < |g16| < 2^-14
     unsigned int pad0[22];
     // line 1: update-kernel accumulators and its work counter (before each
-    // update the counter is zeroed and the last update's stale count moved
-    // into stale_total: by CTA 0 of the check kernel in a whole step, by the
-    // finish in a sharded step)
+    // update CTA 0 of the check kernel zeroes the counter and moves the last
+    // update's stale count into stale_total)
     unsigned long long stale_acc;
     unsigned int upd_next;     // update bins claimed beyond each CTA's first
     unsigned int pad1[29];
-    // line 2: step result, written by the kernel that finishes the step (on
-    // an overflow step of a whole step sumsq is NaN: the check kernel marks
-    // a bin with an inf/NaN gradient that way)
+    // line 2: step result, written by CTA 0 of the update kernel (on an
+    // overflow step of a whole step sumsq is NaN: the check kernel marks a
+    // bin with an inf/NaN gradient that way)
     double sumsq;
     double norm;
     unsigned long long n_nonfinite;
@@ -90,7 +89,7 @@ struct __align__(128) Ctrl {
     unsigned int error;    // checked-mode error bits of both kernels
     float inv_scale;       // binary32 1/S of this step (read by the update)
     float scale_used;      // S of this step
-    // loss-scale state, advanced by the kernel that finishes the step
+    // loss-scale state, advanced by CTA 0 of the update kernel
     float scale;           // S for the next step
     int32_t clean_run;     // consecutive clean steps so far
     unsigned long long steps_total;

@@ -12,9 +12,9 @@
 //                  an overflow step every CTA exits after the sum
 //   refresh_kernel FP16 copy = round-to-nearest-even(master) (Step 1)
 //
-// The sharded step's check pass (mpt_step_partial) instead finishes its own
-// partials by atomic tickets into a 32-byte record, and finish_kernel
-// combines the ranks' records before the update.
+// The sharded step's check pass (mpt_step_partial) instead adds its own
+// partials by atomic tickets into a 32-byte record; the update kernel then
+// adds the ranks' records, in rank order, in place of the partials.
 //
 // All three are HBM-bound streaming kernels on the CUDA cores: there is no
 // contraction, so no tensor-core path.  Per parameter the check reads 2 B and
@@ -66,13 +66,10 @@ struct CheckArgs {
     double host_sq_unscale;  // and 2^(-2e) when S = 2^e, -15 <= e <= 100
     int32_t host_pow2;
     int32_t scale_on_device;  // 1: S is ctrl->scale (asynchronous steps)
-    float clip;           // <= 0: off
-    ScalerParams scaler;
     StatsBlock* stats;    // statistics mode only
-    Partial* partial_out; // sharded step: write this shard's totals here and
-                          // leave the finish to finish_kernel; nullptr: finish
-    int32_t defer_finish; // 1: leave the partials to the update kernel, which
-                          // adds them and finishes the step (whole steps)
+    Partial* partial_out; // sharded step: add the partials into this shard's
+                          // 32-byte record here; nullptr (whole step): leave
+                          // them to the update kernel
 };
 
 struct UpdateArgs {
@@ -85,11 +82,14 @@ struct UpdateArgs {
     float mu;
     float wd;
     float eps;            // Adagrad only
-    // whole steps: the check kernel's partial sums (per bin, or per group of
-    // kFinishGroup bins beyond kOneLevelBins bins), added by every CTA; the
-    // step is finished by CTA 0.  nullptr: the result is already in ctrl.
-    const double* fin_src;
+    // What every CTA adds before it updates; CTA 0 then finishes the step.
+    // Whole step: the check kernel's partial sums (per bin, or per group of
+    // kFinishGroup bins beyond kOneLevelBins bins).  Sharded step: the
+    // ranks' 32-byte records, in rank order.  Exactly one is set.
+    const double* fin_partials;
     int32_t fin_n;
+    const Partial* fin_records;
+    int32_t fin_world;
     int32_t stats_level;  // kNoStats, kMaxOnly or kMaxHist
     float clip;
     ScalerParams scaler;
@@ -125,8 +125,7 @@ __device__ __forceinline__ SqParams sq_params(float S)
 __device__ __forceinline__ void finish_step(Ctrl* c, float S, const SqParams& q,
                                             unsigned long long n_nonfinite, double sumsq,
                                             unsigned int max_mag, bool have_max,
-                                            unsigned int err, float clip, const ScalerParams& sp,
-                                            bool deferred = false)
+                                            unsigned int err, float clip, const ScalerParams& sp)
 {
     const bool found = n_nonfinite != 0;
     const double norm = found ? __longlong_as_double(0x7ff0000000000000ll) : sqrt(sumsq);
@@ -143,17 +142,11 @@ __device__ __forceinline__ void finish_step(Ctrl* c, float S, const SqParams& q,
     c->found_inf = found ? 1 : 0;
     c->clipped = clipped ? 1 : 0;
     c->coef = clipped ? __double2float_rn((double)clip / norm) : 1.0f;
-    if (deferred) {
-        // S, 1/S, the cleared error word, the update's bin counter and the
-        // stale total were set by the check kernel's CTA 0; the update's own
-        // CTAs may be adding error bits right now
-        if (err)
-            atomicOr(&c->error, err);
-    } else {
-        c->inv_scale = q.inv_scale;
-        c->scale_used = S;
-        c->error = err;
-    }
+    // S, 1/S, the cleared error word, the update's bin counter and the stale
+    // total were set by the check kernel's CTA 0; the update's own CTAs may
+    // be adding error bits right now
+    if (err)
+        atomicOr(&c->error, err);
     // Loss-scale state machine: on overflow skip and multiply S by beta;
     // dynamic mode: after growth_interval consecutive clean steps multiply S
     // by alpha; direct mode: S = 65504 / (margin * max|g|) of this step
@@ -184,15 +177,10 @@ __device__ __forceinline__ void finish_step(Ctrl* c, float S, const SqParams& q,
     c->next_pow2 = nq.pow2 ? 1 : 0;
     c->clean_run = clean;
     c->steps_total += 1;
-    // range counts of this step's check pass; in a sharded step also the
-    // previous update's stale count joins the running total and the update's
-    // bin counter starts over (a whole step's check kernel did both already)
+    // range counts of this step's check pass (in a sharded step: of this
+    // rank's shard)
     c->n_zero = atomicExch(&c->zero_acc, 0ull);
     c->n_subnormal = atomicExch(&c->subnormal_acc, 0ull);
-    if (!deferred) {
-        c->stale_total += atomicExch(&c->stale_acc, 0ull);
-        c->upd_next = 0;
-    }
 }
 
 
@@ -662,9 +650,8 @@ __global__ void __launch_bounds__(kThreads, kStats == kMaxHist ? 4 : 8) check_ke
     const Tables& t = a.t;
     const Bin bin = t.bins[blockIdx.x];
     // S of these gradients: the host's, or the device state the previous
-    // step left (written only by the kernel that finishes a step: the update
-    // kernel before this one, or this kernel's last CTA in a sharded step,
-    // after every other CTA has finished reading it)
+    // step left (written only by CTA 0 of the update kernel, which has
+    // completed before this kernel starts)
     float S;
     SqParams q;
     if (a.scale_on_device) {
@@ -679,7 +666,7 @@ __global__ void __launch_bounds__(kThreads, kStats == kMaxHist ? 4 : 8) check_ke
         q.sq_unscale = a.host_sq_unscale;
         q.pow2 = a.host_pow2 != 0;
     }
-    if (a.defer_finish && blockIdx.x == 0 && threadIdx.x == 0) {
+    if (blockIdx.x == 0 && threadIdx.x == 0) {
         // For the update kernel, which finishes this step: S and 1/S of
         // these gradients, a cleared error word, its bin counter at zero, and
         // the last update's stale count moved into the total (that update
@@ -792,7 +779,7 @@ __global__ void __launch_bounds__(kThreads, kStats == kMaxHist ? 4 : 8) check_ke
         // so the total is NaN exactly when the step overflowed (every other
         // partial is in [0, +inf]: +inf only from a binary32 product that a
         // huge 1/S overflowed, and a sum of those is never NaN)
-        a.partials[blockIdx.x] = (a.defer_finish && nf) ? __longlong_as_double(0x7ff8000000000000ll) : part;
+        a.partials[blockIdx.x] = (!a.partial_out && nf) ? __longlong_as_double(0x7ff8000000000000ll) : part;
         if (nf)
             atomicAdd(&a.ctrl->nonfinite_acc, (unsigned long long)nf);
         if (valid) {
@@ -816,7 +803,7 @@ __global__ void __launch_bounds__(kThreads, kStats == kMaxHist ? 4 : 8) check_ke
     // Either way the additions follow a fixed pattern (bin order within a
     // thread's share, a fixed tree across threads), whichever CTA is last.
     __syncthreads();  // every write of this CTA precedes its ticket
-    if (a.defer_finish && (int)gridDim.x <= kOneLevelBins)
+    if (!a.partial_out && (int)gridDim.x <= kOneLevelBins)
         return;  // the update kernel adds the per-bin partials
     double sumsq;
     if ((int)gridDim.x <= kOneLevelBins) {
@@ -844,7 +831,7 @@ __global__ void __launch_bounds__(kThreads, kStats == kMaxHist ? 4 : 8) check_ke
         const double gsum = block_sum(
             threadIdx.x < g_len ? __ldcg(a.partials + g_begin + threadIdx.x) : 0.0, s_red);
         const int ngroups = ((int)gridDim.x + kFinishGroup - 1) / kFinishGroup;
-        if (a.defer_finish) {
+        if (!a.partial_out) {
             // the update kernel adds the group sums
             if (threadIdx.x == 0) {
                 a.group_partials[grp] = gsum;
@@ -865,7 +852,8 @@ __global__ void __launch_bounds__(kThreads, kStats == kMaxHist ? 4 : 8) check_ke
         sumsq = block_sum(sum_partials(a.group_partials, ngroups), s_red);
     }
 
-    // Last CTA: every CTA's partial and counters are visible.
+    // Last CTA of a sharded step's check pass: every CTA's partial and
+    // counters are visible; they become this shard's record.
     Ctrl* c = a.ctrl;
     if constexpr (kStats == kMaxHist) {
         if (threadIdx.x < 32) {
@@ -877,52 +865,13 @@ __global__ void __launch_bounds__(kThreads, kStats == kMaxHist ? 4 : 8) check_ke
         const unsigned int err = atomicExch(&c->error_acc, 0u);
         const unsigned int mm = kStats != kNoStats ? atomicExch(&c->max_mag_acc, 0u) : 0u;
         c->ticket = 0;
-        if (a.partial_out) {
-            // sharded step: the totals of this shard; finish_kernel combines
-            // every rank's record
-            Partial p{};
-            p.sumsq = sumsq;
-            p.n_nonfinite = n_nonfinite;
-            p.max_mag = mm;
-            p.error = err;
-            *a.partial_out = p;
-        } else {
-            finish_step(c, S, q, n_nonfinite, sumsq, mm, kStats != kNoStats, err, a.clip, a.scaler);
-        }
+        Partial p{};
+        p.sumsq = sumsq;
+        p.n_nonfinite = n_nonfinite;
+        p.max_mag = mm;
+        p.error = err;
+        *a.partial_out = p;
     }
-}
-
-// Sharded step: combine the records of all ranks -- in rank order, so every
-// rank obtains bit-identical totals -- and finish the step.  One thread.
-struct FinishArgs {
-    const Partial* parts;  // world records, gathered from every rank
-    int32_t world;
-    int32_t have_max;
-    Ctrl* ctrl;
-    float clip;
-    ScalerParams scaler;
-};
-
-__global__ void finish_kernel(FinishArgs a)
-{
-    if (threadIdx.x != 0 || blockIdx.x != 0)
-        return;
-    double sumsq = 0.0;
-    unsigned long long nf = 0;
-    unsigned int mm = 0, err = 0;
-    for (int r = 0; r < a.world; ++r) {
-        const Partial p = a.parts[r];
-        sumsq += p.sumsq;
-        nf += p.n_nonfinite;
-        mm = max(mm, p.max_mag);
-        err |= p.error;
-    }
-    Ctrl* c = a.ctrl;
-    SqParams q;
-    q.inv_scale = c->next_inv;
-    q.sq_unscale = c->next_sq_unscale;
-    q.pow2 = c->next_pow2 != 0;
-    finish_step(c, c->scale, q, nf, sumsq, mm, a.have_max != 0, err, a.clip, a.scaler);
 }
 
 // ---------------------------------------------------------------------------
@@ -932,6 +881,9 @@ __global__ void finish_kernel(FinishArgs a)
 struct UpdParams {
     float inv_scale, coef, lr, mu, wd, eps;
 };
+
+// Sharded step: ranks' records staged in shared memory per round.
+constexpr int kRecStage = 32;
 
 // Elements of a chunk bin whose master, momentum and gradients the update
 // kernel prefetches into L2 before it waits for the check result.
@@ -1135,6 +1087,7 @@ __global__ void __launch_bounds__(kThreads, kOpt == kOptAdagrad ? 3 : 4) update_
     __shared__ int s_next[2];
     __shared__ unsigned int s_ured[kWarps];
     __shared__ double s_red[kWarps];
+    __shared__ Partial s_rec[kRecStage];
     __shared__ int s_found;
     __shared__ float s_coef;
 
@@ -1170,51 +1123,67 @@ __global__ void __launch_bounds__(kThreads, kOpt == kOptAdagrad ? 3 : 4) update_
     // Wait until the check kernel has finished and its result is visible
     // (returns at once when this grid was launched without overlap).
     asm volatile("griddepcontrol.wait;" ::: "memory");
+    // Add what the check pass left -- the same additions in the same order
+    // in every CTA, so every CTA obtains the same bits -- and derive the
+    // overflow flag, the norm and the clip coefficient.  CTA 0 also finishes
+    // the step: the result, the loss-scale state, the check kernel's
+    // accumulators cleared (this CTA is their only reader).
     Ctrl* c = a.ctrl;
-    float coef;
-    if (a.fin_src) {
-        // Whole step: add the check kernel's partials (the same order of
-        // additions in every CTA, so every CTA obtains the same sum); NaN
-        // means some gradient was inf/NaN.  CTA 0 also finishes the step:
-        // the result, the loss-scale state, the accumulators cleared (this
-        // CTA is their only reader).
-        const double sumsq = block_sum(sum_partials(a.fin_src, a.fin_n), s_red);
-        if (threadIdx.x == 0) {
-            const bool found = isnan(sumsq);
-            const double norm = found ? __longlong_as_double(0x7ff0000000000000ll) : sqrt(sumsq);
-            const bool clipped = !found && a.clip > 0.0f && norm > (double)a.clip;
-            s_found = found ? 1 : 0;
-            s_coef = clipped ? __double2float_rn((double)a.clip / norm) : 1.0f;
-            if (blockIdx.x == 0) {
+    const bool sharded = a.fin_records != nullptr;
+    double sumsq = 0.0;
+    if (!sharded)
+        sumsq = block_sum(sum_partials(a.fin_partials, a.fin_n), s_red);  // valid in thread 0
+    unsigned long long n_nonfinite = 0;
+    unsigned int max_mag = 0, err = 0;
+    if (sharded) {
+        // the ranks' records, added in rank order (as every rank does, so
+        // every rank obtains the same bits), staged 32 at a time
+        for (int base = 0; base < a.fin_world; base += kRecStage) {
+            const int m = min(kRecStage, a.fin_world - base);
+            if ((int)threadIdx.x < m)
+                s_rec[threadIdx.x] = a.fin_records[base + threadIdx.x];
+            __syncthreads();
+            if (threadIdx.x == 0) {
+                for (int r = 0; r < m; ++r) {
+                    sumsq += s_rec[r].sumsq;
+                    n_nonfinite += s_rec[r].n_nonfinite;
+                    max_mag = max(max_mag, s_rec[r].max_mag);
+                    err |= s_rec[r].error;
+                }
+            }
+            __syncthreads();
+        }
+    }
+    if (threadIdx.x == 0) {
+        // whole step: the sum is NaN exactly when some gradient was inf/NaN
+        const bool found = sharded ? n_nonfinite != 0 : isnan(sumsq);
+        const double norm = found ? __longlong_as_double(0x7ff0000000000000ll) : sqrt(sumsq);
+        const bool clipped = !found && a.clip > 0.0f && norm > (double)a.clip;
+        s_found = found ? 1 : 0;
+        s_coef = clipped ? __double2float_rn((double)a.clip / norm) : 1.0f;
+        if (blockIdx.x == 0) {
+            const bool have_max = a.stats_level != kNoStats;
+            if (!sharded) {
+                // (a sharded step's check kernel moved these into its record)
                 if (a.stats_level == kMaxHist)
                     for (int k = 0; k < 32; ++k)
                         a.stats->hist[k] = atomicExch(&a.stats->hist_acc[k], 0ull);
-                const unsigned long long n_nonfinite = atomicExch(&c->nonfinite_acc, 0ull);
-                const unsigned int err = atomicExch(&c->error_acc, 0u);
-                const bool have_max = a.stats_level != kNoStats;
-                const unsigned int mm = have_max ? atomicExch(&c->max_mag_acc, 0u) : 0u;
-                SqParams q;
-                q.inv_scale = __ldcg(&c->inv_scale);
-                q.sq_unscale = 0.0;
-                q.pow2 = false;
-                finish_step(c, __ldcg(&c->scale_used), q, n_nonfinite, sumsq, mm, have_max, err,
-                            a.clip, a.scaler, true);
+                n_nonfinite = atomicExch(&c->nonfinite_acc, 0ull);
+                err = atomicExch(&c->error_acc, 0u);
+                max_mag = have_max ? atomicExch(&c->max_mag_acc, 0u) : 0u;
             }
+            SqParams q;
+            q.inv_scale = __ldcg(&c->inv_scale);
+            q.sq_unscale = 0.0;
+            q.pow2 = false;
+            finish_step(c, __ldcg(&c->scale_used), q, n_nonfinite, sumsq, max_mag, have_max, err,
+                        a.clip, a.scaler);
         }
-        __syncthreads();
-        if (s_found)
-            return;  // Step 6: master, momentum and FP16 copy stay as they are
-        coef = s_coef;
-    } else {
-        // the result finish_kernel left, read past L1 (the hint above may
-        // have cached the line before it was written)
-        if (__ldcg(&c->found_inf) != 0) {
-            // Overflow step (Step 6): master, momentum and FP16 copy stay as
-            // they are.  The flag is the same for every thread of the grid.
-            return;
-        }
-        coef = __ldcg(&c->coef);
     }
+    __syncthreads();
+    if (s_found)
+        return;  // Step 6: master, momentum and FP16 copy stay as they are
+    const float coef = s_coef;
     const UpdParams p{__ldcg(&c->inv_scale), coef, a.lr, a.mu, a.wd, a.eps};
     uint32_t stale = 0;
     bool bad = false;

@@ -103,10 +103,10 @@ def test_emulated_ranks_match_the_whole_step(world):
     (5_000_011, 2048, MPT_FLAG_GRAD_STATS, MPT_SCALER_DIRECT),  # 2 442 bins: two levels
 ])
 def test_whole_step_and_one_rank_sharded_step_agree_bit_for_bit(n, chunk, flags, mode):
-    """A whole step is finished by the update kernel (every CTA adds the check
-    kernel's partials, CTA 0 writes the result and the next S); a one-rank
-    sharded step by the check kernel's ticket finish, its 32-byte record and
-    finish_kernel.  Both add the same partials in the same order, so from the
+    """In a whole step every update CTA adds the check kernel's partials (CTA
+    0 writes the result and the next S); in a one-rank sharded step the check
+    kernel's last CTA adds them into the 32-byte record, and the update adds
+    the one record.  Both add the same partials in the same order, so from the
     same state and gradients they must leave the same bits -- results, loss
     scale, histogram, master, momentum and FP16 copy -- over clean, clipped
     and overflowing steps."""
