@@ -88,6 +88,27 @@ def test_ragged_sample_with_unaligned_pointers_and_injections():
 # edge cases
 # ---------------------------------------------------------------------------
 
+@pytest.mark.parametrize("n", [2048 * 2048, 2048 * 2048 + 1, 2110 * 2048 + 5])
+def test_partial_sum_levels_at_their_boundary(n):
+    """2 048-element check bins over one tensor: exactly 2 048 bins (the
+    largest list whose per-bin partials the update kernel adds directly),
+    2 049 bins (the smallest with sums per group of 64 bins: 33 groups, the
+    last of one bin) and 2 111 bins (a last group of 63).  The check kernel
+    and the host must choose the same level; a clipped, an overflowing and
+    another clipped step match the oracle (bit for bit where the two clip
+    coefficients agree, as everywhere)."""
+    plan = {2: [(0, n - 1, 0x7C00)]}
+    cfg = custom([n], law=("log2_uniform", -26.0, -4.0), scale0=2.0 ** 12, clip=0.05, steps=3,
+                 injections=lambda s: plan.get(s, []))
+    p = Pair(cfg, chunk=2048)
+    found, clipped = [], []
+    for _ in range(cfg.steps):
+        r, _ = p.step()
+        found.append(r["found_inf"])
+        clipped.append(r["clipped"])
+    assert found == [0, 1, 0] and clipped == [1, 0, 1]
+
+
 @pytest.mark.parametrize("sizes", [[1], [2, 3], list(range(1, 18)), [7] * 5000,
                                    [1024, 1025, 1023], [32768], [32769, 32767, 65536 + 5],
                                    [200_003]])
