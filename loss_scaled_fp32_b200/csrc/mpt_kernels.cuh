@@ -177,10 +177,6 @@ __device__ __forceinline__ void finish_step(Ctrl* c, float S, const SqParams& q,
     c->next_pow2 = nq.pow2 ? 1 : 0;
     c->clean_run = clean;
     c->steps_total += 1;
-    // range counts of this step's check pass (in a sharded step: of this
-    // rank's shard)
-    c->n_zero = atomicExch(&c->zero_acc, 0ull);
-    c->n_subnormal = atomicExch(&c->subnormal_acc, 0ull);
 }
 
 
@@ -865,6 +861,11 @@ __global__ void __launch_bounds__(kThreads, kStats == kMaxHist ? 4 : 8) check_ke
         const unsigned int err = atomicExch(&c->error_acc, 0u);
         const unsigned int mm = kStats != kNoStats ? atomicExch(&c->max_mag_acc, 0u) : 0u;
         c->ticket = 0;
+        // this shard's range counts go straight to the result, so that every
+        // accumulator is clear again when the pass ends (a check pass whose
+        // step is never finished leaves nothing for the next step)
+        c->n_zero = atomicExch(&c->zero_acc, 0ull);
+        c->n_subnormal = atomicExch(&c->subnormal_acc, 0ull);
         Partial p{};
         p.sumsq = sumsq;
         p.n_nonfinite = n_nonfinite;
@@ -1164,13 +1165,16 @@ __global__ void __launch_bounds__(kThreads, kOpt == kOptAdagrad ? 3 : 4) update_
         if (blockIdx.x == 0) {
             const bool have_max = a.stats_level != kNoStats;
             if (!sharded) {
-                // (a sharded step's check kernel moved these into its record)
+                // (a sharded step's check kernel moved these into its record
+                // and its result fields)
                 if (a.stats_level == kMaxHist)
                     for (int k = 0; k < 32; ++k)
                         a.stats->hist[k] = atomicExch(&a.stats->hist_acc[k], 0ull);
                 n_nonfinite = atomicExch(&c->nonfinite_acc, 0ull);
                 err = atomicExch(&c->error_acc, 0u);
                 max_mag = have_max ? atomicExch(&c->max_mag_acc, 0u) : 0u;
+                c->n_zero = atomicExch(&c->zero_acc, 0ull);
+                c->n_subnormal = atomicExch(&c->subnormal_acc, 0ull);
             }
             SqParams q;
             q.inv_scale = __ldcg(&c->inv_scale);

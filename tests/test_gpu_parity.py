@@ -10,7 +10,8 @@ import torch
 import oracle
 import workloads as W
 from workloads.configs import Config as WConfig, TensorSpec, miniature
-from loss_scaled_fp32_b200 import MPT, Config, MPT_FLAG_CHECKED, MPT_FLAG_COUNT_STALE
+from loss_scaled_fp32_b200 import (MPT, Config, MPT_FLAG_CHECKED, MPT_FLAG_COUNT_STALE,
+                                   MPT_FLAG_GRAD_STATS)
 
 from parity import Pair
 
@@ -107,6 +108,25 @@ def test_partial_sum_levels_at_their_boundary(n):
         found.append(r["found_inf"])
         clipped.append(r["clipped"])
     assert found == [0, 1, 0] and clipped == [1, 0, 1]
+
+
+def test_an_abandoned_sharded_check_leaves_nothing_for_the_next_step():
+    """A check pass queued by mpt_step_partial whose step is never finished
+    (no mpt_step_finish follows) must leave no count, flag or statistic
+    behind: the whole steps after it match the oracle for their own gradients
+    alone (range counts, non-finite count, histogram, state)."""
+    cfg = custom([70_001, 999, 4097], growth_interval=2, steps=2)
+    p = Pair(cfg, flags=MPT_FLAG_GRAD_STATS)
+    junk = p.grads(9, p.scale)
+    junk[5] = 0x7C00                 # +inf
+    junk[10:200] = 0                 # zeros
+    junk[300:400] = 1                # the smallest subnormal
+    p.flat.copy_(junk)
+    p.opt.step_partial(p.gviews)
+    torch.cuda.synchronize()
+    for _ in range(cfg.steps):
+        r, _ = p.step()
+        assert r["found_inf"] == 0
 
 
 @pytest.mark.parametrize("sizes", [[1], [2, 3], list(range(1, 18)), [7] * 5000,
