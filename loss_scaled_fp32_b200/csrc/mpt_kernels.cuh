@@ -529,7 +529,8 @@ __device__ __forceinline__ CtaTotals block_totals(double x, unsigned int nz, uns
 // increasing i, eight loads issued before they are added (the same order of
 // additions as one load at a time).  Slots past n read as +0.0, which leaves
 // the running sum unchanged: the partials are non-negative, +inf or NaN, so
-// the sum is never -0.0.  The last batch is thereby one round of loads too.
+// the sum is never -0.0.  The last, partly filled batch is thereby issued at
+// once like the others.
 __device__ __forceinline__ double sum_partials(const double* partials, int n)
 {
     constexpr int kU = 8;
