@@ -47,3 +47,15 @@ def test_traffic_figures_only_for_the_current_kernels(tmp_path, monkeypatch):
 def test_l2_note_flags_resident_state():
     assert "L2-resident" in bench.l2_note(1 << 20)
     assert "larger than L2" in bench.l2_note(354_823_168)
+
+
+def test_kernel_digest_ignores_comments_and_layout_only():
+    """The digest that ties stored ncu figures to the device code changes
+    with the code, not with its comments or line breaks."""
+    from loss_scaled_fp32_b200 import build as mbuild
+    a = "int f(int x)\n{\n    return x + 1;  // one more\n}\n"
+    b = "/* a note */ int f(int x) { return x + 1; }"
+    c = "int f(int x)\n{\n    return x + 2;  // one more\n}\n"
+    assert mbuild._code_only(a) == mbuild._code_only(b)
+    assert mbuild._code_only(a) != mbuild._code_only(c)
+    assert len(mbuild.kernel_digest()) == 64
