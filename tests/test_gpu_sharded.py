@@ -18,8 +18,8 @@ import pytest
 import torch
 
 import oracle
-from loss_scaled_fp32_b200 import (MPT, MPT_FLAG_GRAD_STATS, MPT_PARTIAL_BYTES, MPT_SCALER_DIRECT,
-                                   Config, shard_len)
+from loss_scaled_fp32_b200 import (MPT, MPT_FLAG_COUNT_STALE, MPT_FLAG_GRAD_STATS, MPT_PARTIAL_BYTES,
+                                   MPT_SCALER_DIRECT, Config, shard_len)
 
 pytestmark = pytest.mark.gpu
 
@@ -99,7 +99,7 @@ def test_emulated_ranks_match_the_whole_step(world):
 
 
 @pytest.mark.parametrize("n,chunk,flags,mode", [
-    (3_000_017, 0, 0, 0),                                       # 733 check bins: one level
+    (3_000_017, 0, MPT_FLAG_COUNT_STALE, 0),                    # 733 check bins: one level
     (5_000_011, 2048, MPT_FLAG_GRAD_STATS, MPT_SCALER_DIRECT),  # 2 442 bins: two levels
 ])
 def test_whole_step_and_one_rank_sharded_step_agree_bit_for_bit(n, chunk, flags, mode):
@@ -108,8 +108,8 @@ def test_whole_step_and_one_rank_sharded_step_agree_bit_for_bit(n, chunk, flags,
     kernel's last CTA adds them into the 32-byte record, and the update adds
     the one record.  Both add the same partials in the same order, so from the
     same state and gradients they must leave the same bits -- results, loss
-    scale, histogram, master, momentum and FP16 copy -- over clean, clipped
-    and overflowing steps."""
+    scale, histogram, stale counts, master, momentum and FP16 copy -- over
+    clean, clipped and overflowing steps."""
     rng = np.random.default_rng(n)
     master = rng.normal(0, 0.05, n).astype(np.float32)
     cfg = Config(growth_interval=2, check_chunk_elems=chunk, flags=flags, scaler_mode=mode)
@@ -137,7 +137,12 @@ def test_whole_step_and_one_rank_sharded_step_agree_bit_for_bit(n, chunk, flags,
         assert torch.equal(a.w16(0), b.w16(0)), step
         if flags & MPT_FLAG_GRAD_STATS:
             assert a.grad_histogram() == b.grad_histogram(), step
+        sa, sb = a.stats(), b.stats()
+        for k in ("steps", "skipped", "n_fp16_stale_total"):
+            assert sa[k] == sb[k], (step, k)
     assert {"overflow", "clipped"} <= seen
+    if flags & MPT_FLAG_COUNT_STALE:
+        assert a.stats()["n_fp16_stale_total"] > 0
     a.close()
     b.close()
 
